@@ -1,0 +1,165 @@
+/*
+ * libflashspmm: Load-as-Sparse / Compute-as-Dense (LSCD) SpMM for B200 (sm_100a).
+ *
+ * Computes C = A x B where A is an unstructured-pruned fp16 weight matrix
+ * (M x K) held in the Tiled-CSL format and B is a skinny fp16 activation
+ * matrix (K x N, N <= 256), with fp32 accumulation and fp16 output.
+ *
+ * Sources: the Flash-LLM paper review page ("Flash-LLM: Enabling
+ * Cost-Effective and Highly-Efficient Large Generative Model Inference with
+ * Unstructured Sparsity", xllm-io.github.io paper review):
+ *   [core-formulas]  section 3, "core formulas": C = A x B with A in R^{M x K}
+ *                    the sparse weights and B in R^{K x N} the dense features.
+ *   [tiled-csl]      section 3, "sparse encoding format: Tiled-CSL":
+ *                    NonZeros[] grouped by tile, one 32-bit word per nonzero
+ *                    = [16-bit value | 16-bit in-tile index], TileOffsets[]
+ *                    locating each tile, 128-bit vectorised loads.
+ *   [lscd]           section 2, "solution overview": load the weights in
+ *                    sparse form, expand on chip, multiply densely on tensor
+ *                    cores.
+ *   [code-layout]    section 5, "project structure": SpMM_API (host wrapper),
+ *                    SpMM kernel and Reduction kernel (split-K partial sums).
+ *
+ * Format (Tiled-CSL as this library reads it):
+ *   - tiles of tile_m x tile_k, enumerated row-major over the tile grid
+ *     (t = i * ceil(K/tile_k) + j); edge tiles may be ragged;
+ *   - loc = r * tile_k + c inside the tile (row-major, full tile_k pitch);
+ *   - word = fp16 bits | (loc << 16); stored iff the fp16 bits are not 0x0000;
+ *   - words of a tile in ascending loc, padded to a multiple of 4 words with
+ *     the sentinel 0xFFFF0000; tile_m * tile_k <= 65535;
+ *   - tile_offsets: int32[num_tiles + 1], in words, tile_offsets[0] = 0.
+ *
+ * Conventions for every call:
+ *   - Array arguments are DEVICE pointers owned by the caller (the only host
+ *     pointers are B_host / C_host of flashspmm_spmm_lscd_host); the library
+ *     allocates no device memory and keeps no pointer after the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous on that stream.
+ *   - Argument errors detectable on the host return synchronously and launch
+ *     nothing.  Errors found by a kernel (corrupt format, timeout) are recorded
+ *     in a device status word read by flashspmm_get_device_status().
+ *   - No call throws; none synchronises except flashspmm_get_device_status().
+ */
+#ifndef FLASHSPMM_H
+#define FLASHSPMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FLASHSPMM_ABI_VERSION 1
+
+typedef enum {
+  FLASHSPMM_OK = 0,
+  FLASHSPMM_ERR_INVALID_ARG = 1,    /* null pointer, negative size, mismatched view */
+  FLASHSPMM_ERR_UNSUPPORTED = 2,    /* shape or tile outside what the kernels handle */
+  FLASHSPMM_ERR_ALIGNMENT = 3,      /* a pointer or leading dimension breaks 16-byte alignment */
+  FLASHSPMM_ERR_CAPACITY = 4,       /* output buffer / workspace too small, or > 2^31 words */
+  FLASHSPMM_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
+  FLASHSPMM_ERR_CORRUPT_FORMAT = 6, /* tile offsets or words violate the format */
+  FLASHSPMM_ERR_TIMEOUT = 7,        /* a bounded in-kernel wait ran out (kernel exited early) */
+  FLASHSPMM_ERR_NO_DEVICE = 8       /* no usable sm_100 device is current */
+} flashspmm_status;
+
+/* A read-only view of a Tiled-CSL matrix in device memory.  The library owns
+ * nothing it points to. */
+typedef struct {
+  int32_t M, K;                 /* dense shape of A */
+  int32_t tile_m, tile_k;       /* format tile; the SpMM kernel needs 64 x 64 */
+  int64_t nnz;                  /* stored entries excluding padding (informational) */
+  int64_t nwords;               /* == tile_offsets[num_tiles] */
+  const int32_t* tile_offsets;  /* device, num_tiles + 1 entries */
+  const uint32_t* words;        /* device, nwords entries, 16-byte aligned */
+} flashspmm_tcsl;
+
+/* ABI version of the loaded library (FLASHSPMM_ABI_VERSION at build time). */
+int flashspmm_abi_version(void);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char* flashspmm_status_string(int status);
+
+/* Number of format tiles: ceil(M / tile_m) * ceil(K / tile_k); -1 on bad args. */
+int64_t flashspmm_num_tiles(int32_t M, int32_t K, int32_t tile_m, int32_t tile_k);
+
+/* Encoder, pass 1 of 2 [tiled-csl]: counts the nonzero bit patterns of every
+ * tile of A and writes the padded running offsets.
+ *   A             device fp16, M x K row-major, 16-byte aligned, K % 8 == 0.
+ *   tile_m/tile_k tile_m >= 1, tile_k % 8 == 0, tile_m * tile_k <= 65535.
+ *   tile_offsets  device int32[num_tiles + 1]; receives the Tiled-CSL offsets.
+ *   nnz           device int64[1]; receives the number of stored entries.
+ * Read tile_offsets[num_tiles] (the word count) after the stream reaches this
+ * point to size the words buffer for pass 2.  A total above 2^31 - 1 words
+ * records FLASHSPMM_ERR_CAPACITY in the device status word. */
+flashspmm_status flashspmm_tcsl_count(const void* A, int32_t M, int32_t K, int32_t tile_m, int32_t tile_k,
+                                      int32_t* tile_offsets, int64_t* nnz, void* stream);
+
+/* Encoder, pass 2 of 2 [tiled-csl]: writes every tile's words in ascending loc
+ * followed by sentinel padding, at the offsets from pass 1.  Output is
+ * bit-identical to the format definition above.
+ *   words           device uint32[words_capacity], 16-byte aligned.
+ * A tile whose entries do not fit its offset range (A changed since pass 1) or
+ * an offset beyond words_capacity records FLASHSPMM_ERR_CAPACITY and that tile
+ * is left unwritten. */
+flashspmm_status flashspmm_tcsl_fill(const void* A, int32_t M, int32_t K, int32_t tile_m, int32_t tile_k,
+                                     const int32_t* tile_offsets, uint32_t* words, int64_t words_capacity,
+                                     void* stream);
+
+/* Checked mode: verifies a Tiled-CSL view on the GPU (offsets start at 0,
+ * non-decreasing, multiples of 4, end at nwords, segment <= roundup4(area);
+ * each tile holds real words in strictly ascending in-range loc with nonzero
+ * value bits, then only exact sentinels).  Any violation records
+ * FLASHSPMM_ERR_CORRUPT_FORMAT in the device status word. */
+flashspmm_status flashspmm_tcsl_validate(const flashspmm_tcsl* A, void* stream);
+
+/* Bytes of workspace flashspmm_spmm_lscd needs on the CURRENT device for this
+ * problem (0 when no partial sums are needed).  split_k as below. */
+size_t flashspmm_spmm_workspace_bytes(int32_t M, int32_t K, int32_t N, int32_t split_k);
+
+/* LSCD SpMM [lscd][core-formulas]: C = A x B.
+ *   A          Tiled-CSL view with tile_m = tile_k = 64; A->M == M, A->K == K.
+ *   B          device fp16, K x N column-major (a contiguous [N][K] array),
+ *              16-byte aligned, K % 8 == 0.  B must be finite: the product is
+ *              computed densely per tile, so a non-finite B value meets the
+ *              tile's stored zeros.
+ *   C          device fp16, M x N column-major (a contiguous [N][M] array).
+ *   N          1 <= N <= 256.
+ *   split_k    0: automatic, the step space (units of 128 rows x 64-wide K
+ *              tiles) is cut into one contiguous piece per SM and units shared
+ *              by several pieces are reduced by the last CTA to finish
+ *              ([code-layout] Reduction kernel, fused here); >= 1: each
+ *              128-row unit is cut into min(split_k, ceil(K/64)) K-chunks.
+ *              Results are deterministic for a given (problem, split_k, device).
+ *   workspace  device, >= flashspmm_spmm_workspace_bytes(...), 16-byte aligned;
+ *              may be NULL when that size is 0.  Holds fp32 partial sums and
+ *              per-unit arrival counters; it is cleared by the call itself.
+ * K == 0 writes zeros to C; M == 0 or N == 0 does nothing. */
+flashspmm_status flashspmm_spmm_lscd(const flashspmm_tcsl* A, const void* B, void* C, int32_t M, int32_t K,
+                                     int32_t N, int32_t split_k, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
+/* End-to-end form of flashspmm_spmm_lscd for callers whose activations live
+ * in host memory: on `stream` it copies B from B_host (K x N column-major fp16)
+ * into the caller's device staging buffer B_dev, runs the SpMM into the
+ * device buffer C_dev, and copies C back to C_host (M x N column-major fp16).
+ * Host buffers should be pinned for the copies to overlap; the call returns
+ * before the copies finish.  Same argument rules as flashspmm_spmm_lscd. */
+flashspmm_status flashspmm_spmm_lscd_host(const flashspmm_tcsl* A, const void* B_host, void* C_host, void* B_dev,
+                                          void* C_dev, int32_t M, int32_t K, int32_t N, int32_t split_k,
+                                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the library's device status
+ * word for the current device: FLASHSPMM_OK or the first error a kernel
+ * recorded since the last read. */
+flashspmm_status flashspmm_get_device_status(void* stream);
+
+/* Number of kernels this library has launched in this process (diagnostic). */
+uint64_t flashspmm_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLASHSPMM_H */

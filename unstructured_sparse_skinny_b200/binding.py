@@ -1,0 +1,209 @@
+"""ctypes binding of libflashspmm (argument marshalling only).
+
+Names follow the C ABI in ``include/flashspmm.h`` and the problem statement of
+the Flash-LLM review (section 3, "core formulas": C = A x B with sparse
+weights A and dense features B): ``tcsl_encode(A_dense, tile_m, tile_k)`` and
+``spmm_lscd(tcsl_A, B, C, M, K, N, split_k, stream)``.
+
+Layouts: A is a row-major ``[M, K]`` fp16 tensor; B is passed as the
+contiguous ``[N, K]`` tensor (K x N column-major); C is returned as the
+contiguous ``[N, M]`` tensor (M x N column-major).
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from pathlib import Path
+
+import torch
+
+_PKG = Path(__file__).resolve().parent
+_LIB_PATH = _PKG / "libflashspmm.so"
+_lib = None
+
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "ALIGNMENT", 4: "CAPACITY", 5: "CUDA",
+                6: "CORRUPT_FORMAT", 7: "TIMEOUT", 8: "NO_DEVICE"}
+
+
+class FlashSpmmError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS_NAMES.get(self.status, self.status)} "
+                         f"({_lib.flashspmm_status_string(self.status).decode() if _lib else ''})")
+
+
+class _TcslView(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int32), ("K", ctypes.c_int32), ("tile_m", ctypes.c_int32),
+                ("tile_k", ctypes.c_int32), ("nnz", ctypes.c_int64), ("nwords", ctypes.c_int64),
+                ("tile_offsets", ctypes.c_void_p), ("words", ctypes.c_void_p)]
+
+
+def load_library():
+    """Load libflashspmm.so from the package directory (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not _LIB_PATH.exists():
+        raise RuntimeError(f"{_LIB_PATH} is missing: build it with `python -m unstructured_sparse_skinny_b200.build`"
+                           " (the library has no CPU fallback)")
+    lib = ctypes.CDLL(str(_LIB_PATH))
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    VP = ctypes.POINTER(_TcslView)
+    sig = {
+        "flashspmm_abi_version": (ctypes.c_int, []),
+        "flashspmm_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "flashspmm_num_tiles": (I64, [I32, I32, I32, I32]),
+        "flashspmm_tcsl_count": (ctypes.c_int, [P, I32, I32, I32, I32, P, P, P]),
+        "flashspmm_tcsl_fill": (ctypes.c_int, [P, I32, I32, I32, I32, P, P, I64, P]),
+        "flashspmm_tcsl_validate": (ctypes.c_int, [VP, P]),
+        "flashspmm_spmm_workspace_bytes": (SZ, [I32, I32, I32, I32]),
+        "flashspmm_spmm_lscd": (ctypes.c_int, [VP, P, P, I32, I32, I32, I32, P, SZ, P]),
+        "flashspmm_spmm_lscd_host": (ctypes.c_int, [VP, P, P, P, P, I32, I32, I32, I32, P, SZ, P]),
+        "flashspmm_get_device_status": (ctypes.c_int, [P]),
+        "flashspmm_launch_count": (ctypes.c_uint64, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype, f.argtypes = res, args
+    _lib = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise FlashSpmmError(status, where)
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+@dataclass
+class TCSL:
+    """A Tiled-CSL matrix resident in device memory."""
+    tile_offsets: torch.Tensor  # int32 [num_tiles + 1]
+    words: torch.Tensor         # int32 storage of the uint32 words [nwords]
+    nnz: int
+    M: int
+    K: int
+    tile_m: int = 64
+    tile_k: int = 64
+
+    @property
+    def nwords(self) -> int:
+        return int(self.words.numel())
+
+    def view(self) -> _TcslView:
+        return _TcslView(self.M, self.K, self.tile_m, self.tile_k, self.nnz, self.nwords,
+                         self.tile_offsets.data_ptr(), self.words.data_ptr() if self.nwords else None)
+
+
+def tcsl_encode(A_dense: torch.Tensor, tile_m: int = 64, tile_k: int = 64, stream=None) -> TCSL:
+    """Encode a row-major fp16 ``[M, K]`` device tensor into Tiled-CSL on the GPU.
+
+    Runs the count pass, reads the word total back (one host sync), allocates
+    the words with torch, then runs the fill pass."""
+    lib = load_library()
+    if A_dense.dtype != torch.float16 or A_dense.dim() != 2 or not A_dense.is_cuda:
+        raise TypeError("A_dense must be a 2-D float16 CUDA tensor")
+    A = A_dense.contiguous()
+    M, K = A.shape
+    s = _stream_handle(stream)
+    nt = lib.flashspmm_num_tiles(M, K, tile_m, tile_k)
+    if nt < 0:
+        raise FlashSpmmError(1, "tcsl_encode")
+    off = torch.empty(nt + 1, dtype=torch.int32, device=A.device)
+    nnz = torch.empty(1, dtype=torch.int64, device=A.device)
+    _check(lib.flashspmm_tcsl_count(A.data_ptr() if A.numel() else None, M, K, tile_m, tile_k,
+                                    off.data_ptr(), nnz.data_ptr(), s), "tcsl_count")
+    _check(lib.flashspmm_get_device_status(s), "tcsl_count (device)")  # synchronises the stream
+    nwords = int(off[-1].item())
+    words = torch.empty(max(nwords, 0), dtype=torch.int32, device=A.device)
+    _check(lib.flashspmm_tcsl_fill(A.data_ptr() if A.numel() else None, M, K, tile_m, tile_k, off.data_ptr(),
+                                   words.data_ptr() if nwords else None, nwords, s), "tcsl_fill")
+    return TCSL(off, words, int(nnz.item()), M, K, tile_m, tile_k)
+
+
+def tcsl_validate(A: TCSL, stream=None) -> None:
+    """Checked mode: raises FlashSpmmError(CORRUPT_FORMAT) if the encoding is invalid."""
+    lib = load_library()
+    s = _stream_handle(stream)
+    v = A.view()
+    _check(lib.flashspmm_tcsl_validate(ctypes.byref(v), s), "tcsl_validate")
+    _check(lib.flashspmm_get_device_status(s), "tcsl_validate (device)")
+
+
+def spmm_workspace_bytes(M: int, K: int, N: int, split_k: int = 0) -> int:
+    return int(load_library().flashspmm_spmm_workspace_bytes(M, K, N, split_k))
+
+
+_workspaces: dict = {}
+
+
+def _workspace(device: torch.device, nbytes: int) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    key = (device.index, )
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def spmm_lscd(tcsl_A: TCSL, B: torch.Tensor, C: torch.Tensor | None = None, M: int | None = None,
+              K: int | None = None, N: int | None = None, split_k: int = 0, stream=None,
+              workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """C = A x B.  B is the contiguous ``[N, K]`` fp16 tensor; returns C as ``[N, M]`` fp16."""
+    lib = load_library()
+    M = tcsl_A.M if M is None else M
+    K = tcsl_A.K if K is None else K
+    if B.dtype != torch.float16 or B.dim() != 2 or not B.is_cuda or not B.is_contiguous():
+        raise TypeError("B must be a contiguous [N, K] float16 CUDA tensor")
+    N = B.shape[0] if N is None else N
+    if B.shape != (N, K):
+        raise ValueError(f"B has shape {tuple(B.shape)}, expected ({N}, {K})")
+    if C is None:
+        C = torch.empty((N, M), dtype=torch.float16, device=B.device)
+    elif C.shape != (N, M) or C.dtype != torch.float16 or not C.is_contiguous():
+        raise ValueError("C must be a contiguous [N, M] float16 tensor")
+    need = int(lib.flashspmm_spmm_workspace_bytes(M, K, N, split_k))
+    if workspace is None:
+        workspace = _workspace(B.device, need)
+    v = tcsl_A.view()
+    _check(lib.flashspmm_spmm_lscd(ctypes.byref(v), B.data_ptr(), C.data_ptr(), M, K, N, split_k,
+                                   workspace.data_ptr() if workspace is not None else None,
+                                   workspace.numel() if workspace is not None else 0, _stream_handle(stream)),
+           "spmm_lscd")
+    return C
+
+
+def spmm_lscd_host(tcsl_A: TCSL, B_host: torch.Tensor, C_host: torch.Tensor, B_dev: torch.Tensor,
+                   C_dev: torch.Tensor, split_k: int = 0, stream=None,
+                   workspace: torch.Tensor | None = None) -> None:
+    """End-to-end call with host activations: H2D copy of B, SpMM, D2H copy of C (all async on stream)."""
+    lib = load_library()
+    N, K = B_host.shape
+    M = tcsl_A.M
+    need = int(lib.flashspmm_spmm_workspace_bytes(M, K, N, split_k))
+    if workspace is None:
+        workspace = _workspace(B_dev.device, need)
+    v = tcsl_A.view()
+    _check(lib.flashspmm_spmm_lscd_host(ctypes.byref(v), B_host.data_ptr(), C_host.data_ptr(), B_dev.data_ptr(),
+                                        C_dev.data_ptr(), M, K, N, split_k,
+                                        workspace.data_ptr() if workspace is not None else None,
+                                        workspace.numel() if workspace is not None else 0,
+                                        _stream_handle(stream)), "spmm_lscd_host")
+
+
+def check_device_status(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel recorded an error."""
+    _check(load_library().flashspmm_get_device_status(_stream_handle(stream)), "device status")
+
+
+def launch_count() -> int:
+    return int(load_library().flashspmm_launch_count())

@@ -1,0 +1,189 @@
+// extern "C" entry points of libflashspmm: argument checks, then the kernel
+// launchers.  This is the host wrapper the Flash-LLM review lists as
+// SpMM_API (section 5, "project structure"), reshaped as a plain C ABI that
+// takes device pointers, sizes and a stream and never allocates.
+#include <atomic>
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace flashspmm {
+
+__device__ int g_device_status = 0;
+
+static std::atomic<uint64_t> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+int* device_status_ptr() {
+  static std::atomic<int*> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  int* p = cache[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_device_status) != cudaSuccess) return nullptr;
+    p = static_cast<int*>(a);
+    cache[dev].store(p, std::memory_order_release);
+  }
+  return p;
+}
+
+}  // namespace flashspmm
+
+using namespace flashspmm;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+flashspmm_status check_encoder_args(const void* A, int32_t M, int32_t K, int32_t tile_m, int32_t tile_k) {
+  if (M < 0 || K < 0 || tile_m <= 0 || tile_k <= 0) return FLASHSPMM_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(tile_m) * tile_k > 65535) return FLASHSPMM_ERR_UNSUPPORTED;
+  if (tile_k % 8 != 0 || K % 8 != 0) return FLASHSPMM_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(M) * K > 0 && A == nullptr) return FLASHSPMM_ERR_INVALID_ARG;
+  if (A && !aligned16(A)) return FLASHSPMM_ERR_ALIGNMENT;
+  return FLASHSPMM_OK;
+}
+
+flashspmm_status check_view(const flashspmm_tcsl* A) {
+  if (!A) return FLASHSPMM_ERR_INVALID_ARG;
+  if (A->M < 0 || A->K < 0 || A->tile_m <= 0 || A->tile_k <= 0 || A->nwords < 0 || A->nwords > INT32_MAX)
+    return FLASHSPMM_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(A->tile_m) * A->tile_k > 65535) return FLASHSPMM_ERR_UNSUPPORTED;
+  if (!A->tile_offsets) return FLASHSPMM_ERR_INVALID_ARG;
+  if (A->nwords > 0 && !A->words) return FLASHSPMM_ERR_INVALID_ARG;
+  if (A->words && !aligned16(A->words)) return FLASHSPMM_ERR_ALIGNMENT;
+  if ((A->nwords & 3) != 0) return FLASHSPMM_ERR_CORRUPT_FORMAT;
+  return FLASHSPMM_OK;
+}
+
+bool have_device() {
+  int n = 0;
+  return cudaGetDeviceCount(&n) == cudaSuccess && n > 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+int flashspmm_abi_version(void) { return FLASHSPMM_ABI_VERSION; }
+
+const char* flashspmm_status_string(int status) {
+  switch (status) {
+    case FLASHSPMM_OK: return "ok";
+    case FLASHSPMM_ERR_INVALID_ARG: return "invalid argument";
+    case FLASHSPMM_ERR_UNSUPPORTED: return "unsupported shape or tile";
+    case FLASHSPMM_ERR_ALIGNMENT: return "pointer or leading dimension not 16-byte aligned";
+    case FLASHSPMM_ERR_CAPACITY: return "buffer or workspace too small";
+    case FLASHSPMM_ERR_CUDA: return "CUDA runtime error";
+    case FLASHSPMM_ERR_CORRUPT_FORMAT: return "corrupt Tiled-CSL data";
+    case FLASHSPMM_ERR_TIMEOUT: return "bounded in-kernel wait timed out";
+    case FLASHSPMM_ERR_NO_DEVICE: return "no usable CUDA device";
+    default: return "unknown status";
+  }
+}
+
+int64_t flashspmm_num_tiles(int32_t M, int32_t K, int32_t tile_m, int32_t tile_k) {
+  if (M < 0 || K < 0 || tile_m <= 0 || tile_k <= 0) return -1;
+  return static_cast<int64_t>((M + tile_m - 1) / tile_m) * ((K + tile_k - 1) / tile_k);
+}
+
+flashspmm_status flashspmm_tcsl_count(const void* A, int32_t M, int32_t K, int32_t tile_m, int32_t tile_k,
+                                      int32_t* tile_offsets, int64_t* nnz, void* stream) {
+  flashspmm_status st = check_encoder_args(A, M, K, tile_m, tile_k);
+  if (st != FLASHSPMM_OK) return st;
+  if (!tile_offsets || !nnz) return FLASHSPMM_ERR_INVALID_ARG;
+  if (!have_device()) return FLASHSPMM_ERR_NO_DEVICE;
+  return launch_tcsl_count(A, M, K, tile_m, tile_k, tile_offsets, nnz, as_stream(stream)) == cudaSuccess
+             ? FLASHSPMM_OK
+             : FLASHSPMM_ERR_CUDA;
+}
+
+flashspmm_status flashspmm_tcsl_fill(const void* A, int32_t M, int32_t K, int32_t tile_m, int32_t tile_k,
+                                     const int32_t* tile_offsets, uint32_t* words, int64_t words_capacity,
+                                     void* stream) {
+  flashspmm_status st = check_encoder_args(A, M, K, tile_m, tile_k);
+  if (st != FLASHSPMM_OK) return st;
+  if (!tile_offsets || words_capacity < 0 || (words_capacity > 0 && !words)) return FLASHSPMM_ERR_INVALID_ARG;
+  if (words && !aligned16(words)) return FLASHSPMM_ERR_ALIGNMENT;
+  if (!have_device()) return FLASHSPMM_ERR_NO_DEVICE;
+  return launch_tcsl_fill(A, M, K, tile_m, tile_k, tile_offsets, words, words_capacity, as_stream(stream)) ==
+                 cudaSuccess
+             ? FLASHSPMM_OK
+             : FLASHSPMM_ERR_CUDA;
+}
+
+flashspmm_status flashspmm_tcsl_validate(const flashspmm_tcsl* A, void* stream) {
+  flashspmm_status st = check_view(A);
+  if (st != FLASHSPMM_OK) return st;
+  if (!have_device()) return FLASHSPMM_ERR_NO_DEVICE;
+  return launch_tcsl_validate(A, as_stream(stream)) == cudaSuccess ? FLASHSPMM_OK : FLASHSPMM_ERR_CUDA;
+}
+
+size_t flashspmm_spmm_workspace_bytes(int32_t M, int32_t K, int32_t N, int32_t split_k) {
+  if (M <= 0 || K <= 0 || N <= 0 || N > 256) return 0;
+  return make_spmm_plan(M, K, N, split_k, device_sm_count()).workspace_bytes;
+}
+
+flashspmm_status flashspmm_spmm_lscd(const flashspmm_tcsl* A, const void* B, void* C, int32_t M, int32_t K,
+                                     int32_t N, int32_t split_k, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  flashspmm_status st = check_view(A);
+  if (st != FLASHSPMM_OK) return st;
+  if (M < 0 || K < 0 || N < 0 || A->M != M || A->K != K) return FLASHSPMM_ERR_INVALID_ARG;
+  if (A->tile_m != 64 || A->tile_k != 64) return FLASHSPMM_ERR_UNSUPPORTED;
+  if (N > 256 || K % 8 != 0) return FLASHSPMM_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return FLASHSPMM_OK;
+  if (!C) return FLASHSPMM_ERR_INVALID_ARG;
+  if (!have_device()) return FLASHSPMM_ERR_NO_DEVICE;
+  cudaStream_t s = as_stream(stream);
+  if (K == 0) {
+    return cudaMemsetAsync(C, 0, static_cast<size_t>(M) * N * 2, s) == cudaSuccess ? FLASHSPMM_OK
+                                                                                    : FLASHSPMM_ERR_CUDA;
+  }
+  if (!B) return FLASHSPMM_ERR_INVALID_ARG;
+  if (!aligned16(B)) return FLASHSPMM_ERR_ALIGNMENT;
+  const int sms = device_sm_count();
+  if (sms <= 0) return FLASHSPMM_ERR_NO_DEVICE;
+  const SpmmPlan plan = make_spmm_plan(M, K, N, split_k, sms);
+  if (plan.workspace_bytes > 0) {
+    if (!workspace || workspace_bytes < plan.workspace_bytes) return FLASHSPMM_ERR_CAPACITY;
+    if (!aligned16(workspace)) return FLASHSPMM_ERR_ALIGNMENT;
+  }
+  return launch_spmm_lscd(A, B, C, M, K, N, plan, workspace, s);
+}
+
+flashspmm_status flashspmm_spmm_lscd_host(const flashspmm_tcsl* A, const void* B_host, void* C_host, void* B_dev,
+                                          void* C_dev, int32_t M, int32_t K, int32_t N, int32_t split_k,
+                                          void* workspace, size_t workspace_bytes, void* stream) {
+  if (M < 0 || K < 0 || N < 0) return FLASHSPMM_ERR_INVALID_ARG;
+  const size_t b_bytes = static_cast<size_t>(K) * N * 2, c_bytes = static_cast<size_t>(M) * N * 2;
+  if ((b_bytes && (!B_host || !B_dev)) || (c_bytes && (!C_host || !C_dev))) return FLASHSPMM_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  if (b_bytes && cudaMemcpyAsync(B_dev, B_host, b_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return FLASHSPMM_ERR_CUDA;
+  const flashspmm_status st = flashspmm_spmm_lscd(A, B_dev, C_dev, M, K, N, split_k, workspace, workspace_bytes,
+                                                  stream);
+  if (st != FLASHSPMM_OK) return st;
+  if (c_bytes && cudaMemcpyAsync(C_host, C_dev, c_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return FLASHSPMM_ERR_CUDA;
+  return FLASHSPMM_OK;
+}
+
+flashspmm_status flashspmm_get_device_status(void* stream) {
+  if (!have_device()) return FLASHSPMM_ERR_NO_DEVICE;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return FLASHSPMM_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return FLASHSPMM_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return FLASHSPMM_ERR_CUDA;
+  }
+  return static_cast<flashspmm_status>(v);
+}
+
+uint64_t flashspmm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

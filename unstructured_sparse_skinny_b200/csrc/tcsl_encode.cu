@@ -1,0 +1,276 @@
+// GPU Tiled-CSL encoder (Flash-LLM paper review, section 3, "sparse encoding
+// format: Tiled-CSL"): the nonzeros of every tile are stored together as
+// 32-bit [16-bit value | 16-bit in-tile index] words and TileOffsets[] locates
+// each tile.  The pages describe the encoding as an offline step; here it runs
+// as three HBM-bound kernels whose output is bit-identical to the format's
+// definition (ascending loc inside a tile, lists padded to 16 bytes with the
+// sentinel 0xFFFF0000, offsets in words):
+//   1. count:    one warp per tile counts nonzero fp16 bit patterns;
+//   2. scan:     one CTA turns counts into padded running offsets and sums nnz;
+//   3. fill:     one warp per tile compacts the tile in loc order with a warp
+//                prefix sum (no atomics, so positions are deterministic).
+// A fourth kernel validates a given encoding (checked mode).
+#include "common.cuh"
+#include "sm100_primitives.cuh"
+
+namespace flashspmm {
+namespace {
+
+constexpr int kEncThreads = 256;
+constexpr int kWarpsPerBlock = kEncThreads / 32;
+
+__device__ __forceinline__ int nonzero_halves(uint32_t w) {
+  return static_cast<int>((w & 0xFFFFu) != 0u) + static_cast<int>((w >> 16) != 0u);
+}
+
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+struct TileGeom {
+  int64_t row0, col0;  // tile origin in A
+  int rows, cols;      // valid extent (ragged at the matrix edge)
+  int chunks_per_row;  // cols / 8 (16-byte chunks)
+};
+
+__device__ __forceinline__ TileGeom tile_geom(int64_t t, int TK, int M, int K, int tile_m, int tile_k) {
+  TileGeom g;
+  const int64_t i = t / TK, j = t - (t / TK) * TK;
+  g.row0 = i * tile_m;
+  g.col0 = j * tile_k;
+  g.rows = static_cast<int>(min64(tile_m, M - g.row0));
+  g.cols = static_cast<int>(min64(tile_k, K - g.col0));
+  g.chunks_per_row = g.cols >> 3;
+  return g;
+}
+
+// Pass 1: true nonzero count of tile t -> tile_offsets[t + 1].
+__global__ void __launch_bounds__(kEncThreads) tcsl_count_kernel(const uint4* __restrict__ A, int M, int K,
+                                                                int tile_m, int tile_k, int TK,
+                                                                int64_t num_tiles, int32_t* __restrict__ off) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kEncThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarpsPerBlock;
+  const int64_t row_chunks = K >> 3;
+  for (int64_t t = warp0; t < num_tiles; t += nwarps) {
+    const TileGeom g = tile_geom(t, TK, M, K, tile_m, tile_k);
+    const int nchunks = g.rows * g.chunks_per_row;
+    const uint4* base = A + g.row0 * row_chunks + (g.col0 >> 3);
+    int cnt = 0;
+    for (int e = lane; e < nchunks; e += 32) {
+      const int r = e / g.chunks_per_row, ch = e - r * g.chunks_per_row;
+      const uint4 v = __ldg(base + r * row_chunks + ch);
+      cnt += nonzero_halves(v.x) + nonzero_halves(v.y) + nonzero_halves(v.z) + nonzero_halves(v.w);
+    }
+    cnt = warp_sum(cnt);
+    if (lane == 0) off[t + 1] = cnt;
+  }
+}
+
+// Pass 2 (one CTA): tile_offsets[t + 1] <- sum_{t' <= t} roundup4(count_t'),
+// tile_offsets[0] <- 0, *nnz <- sum count_t.
+constexpr int kScanThreads = 1024;
+__global__ void __launch_bounds__(kScanThreads) tcsl_scan_kernel(int32_t* __restrict__ off, int64_t num_tiles,
+                                                                int64_t* __restrict__ nnz, int* status) {
+  __shared__ int64_t s_pad[kScanThreads];
+  __shared__ int64_t s_true[kScanThreads];
+  const int tid = threadIdx.x;
+  const int64_t chunk = (num_tiles + kScanThreads - 1) / kScanThreads;
+  const int64_t b = min64(num_tiles, tid * chunk), e = min64(num_tiles, b + chunk);
+  int64_t pad = 0, tru = 0;
+  for (int64_t i = b; i < e; ++i) {
+    const int32_t c = off[i + 1];
+    tru += c;
+    pad += (c + 3) & ~3;
+  }
+  s_pad[tid] = pad;
+  s_true[tid] = tru;
+  __syncthreads();
+  for (int d = 1; d < kScanThreads; d <<= 1) {  // inclusive Hillis-Steele scan
+    const int64_t x = tid >= d ? s_pad[tid - d] : 0;
+    const int64_t y = tid >= d ? s_true[tid - d] : 0;
+    __syncthreads();
+    s_pad[tid] += x;
+    s_true[tid] += y;
+    __syncthreads();
+  }
+  const int64_t total = s_pad[kScanThreads - 1];
+  if (tid == 0) {
+    off[0] = 0;
+    *nnz = s_true[kScanThreads - 1];
+    if (total > INT32_MAX) record_status(status, FLASHSPMM_ERR_CAPACITY);
+  }
+  int64_t run = s_pad[tid] - pad;
+  for (int64_t i = b; i < e; ++i) {
+    const int32_t c = off[i + 1];
+    run += (c + 3) & ~3;
+    off[i + 1] = static_cast<int32_t>(min64(run, INT32_MAX));
+  }
+}
+
+// Pass 3: words of tile t in ascending loc, then sentinel padding.
+__global__ void __launch_bounds__(kEncThreads) tcsl_fill_kernel(const uint4* __restrict__ A, int M, int K,
+                                                               int tile_m, int tile_k, int TK, int64_t num_tiles,
+                                                               const int32_t* __restrict__ off,
+                                                               uint32_t* __restrict__ words, int64_t capacity,
+                                                               int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kEncThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarpsPerBlock;
+  const int64_t row_chunks = K >> 3;
+  for (int64_t t = warp0; t < num_tiles; t += nwarps) {
+    const int64_t w0 = off[t], w1 = off[t + 1];
+    if (w0 < 0 || w1 < w0 || w1 > capacity || (w0 & 3) || ((w1 - w0) & 3)) {
+      if (lane == 0) record_status(status, FLASHSPMM_ERR_CAPACITY);
+      continue;
+    }
+    const int room = static_cast<int>(w1 - w0);
+    uint32_t* dst = words + w0;
+    const TileGeom g = tile_geom(t, TK, M, K, tile_m, tile_k);
+    const int nchunks = g.rows * g.chunks_per_row;
+    const uint4* base = A + g.row0 * row_chunks + (g.col0 >> 3);
+    int carry = 0;
+    bool overflow = false;
+    for (int e0 = 0; e0 < nchunks; e0 += 32) {
+      const int e = e0 + lane;
+      uint32_t h[4] = {0u, 0u, 0u, 0u};
+      uint32_t loc0 = 0;
+      if (e < nchunks) {
+        const int r = e / g.chunks_per_row, ch = e - r * g.chunks_per_row;
+        const uint4 v = __ldg(base + r * row_chunks + ch);
+        h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w;
+        loc0 = static_cast<uint32_t>(r * tile_k + ch * 8);
+      }
+      uint32_t mask = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t half = (h[k >> 1] >> ((k & 1) * 16)) & 0xFFFFu;
+        mask |= (half != 0u ? 1u : 0u) << k;
+      }
+      const int cnt = __popc(mask);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int pos = carry + incl - cnt;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (mask & (1u << k)) {
+          const uint32_t half = (h[k >> 1] >> ((k & 1) * 16)) & 0xFFFFu;
+          if (pos < room) dst[pos] = half | ((loc0 + k) << 16);
+          else overflow = true;
+          ++pos;
+        }
+      }
+      carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+    const int padded = (carry + 3) & ~3;
+    if (padded != room) overflow = true;
+    for (int q = carry + lane; q < min(padded, room); q += 32) dst[q] = kSentinel;
+    if (__any_sync(0xFFFFFFFFu, overflow) && lane == 0) record_status(status, FLASHSPMM_ERR_CAPACITY);
+  }
+}
+
+// Checked mode: one warp per tile verifies the offsets and the words.
+__global__ void __launch_bounds__(kEncThreads) tcsl_validate_kernel(const int32_t* __restrict__ off,
+                                                                   const uint32_t* __restrict__ words,
+                                                                   int64_t nwords, int M, int K, int tile_m,
+                                                                   int tile_k, int TK, int64_t num_tiles, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kEncThreads + threadIdx.x) >> 5;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarpsPerBlock;
+  const int area = tile_m * tile_k;
+  const int max_words = (area + 3) & ~3;
+  for (int64_t t = warp0; t < num_tiles; t += nwarps) {
+    const int64_t w0 = off[t], w1 = off[t + 1];
+    bool bad = w0 < 0 || w1 < w0 || (w0 & 3) || (w1 & 3) || w1 > nwords || (w1 - w0) > max_words;
+    if (t == 0 && w0 != 0) bad = true;
+    if (t == num_tiles - 1 && w1 != nwords) bad = true;
+    if (bad) {
+      if (lane == 0) record_status(status, FLASHSPMM_ERR_CORRUPT_FORMAT);
+      continue;
+    }
+    const TileGeom g = tile_geom(t, TK, M, K, tile_m, tile_k);
+    int prev_loc = -1;          // last real loc of the previous batch
+    bool seen_sentinel = false;  // a sentinel appeared in an earlier batch
+    int nreal = 0;
+    for (int64_t b0 = w0; b0 < w1; b0 += 32) {
+      const int64_t idx = b0 + lane;
+      const bool valid = idx < w1;
+      const uint32_t w = valid ? words[idx] : kSentinel;
+      const int loc = static_cast<int>(w >> 16);
+      const bool sent = loc == 0xFFFF;
+      bool lane_bad = false;
+      if (valid && sent && w != kSentinel) lane_bad = true;
+      if (valid && !sent) {
+        const int r = loc / tile_k, c = loc - (loc / tile_k) * tile_k;
+        if (loc >= area || r >= g.rows || c >= g.cols || (w & 0xFFFFu) == 0u) lane_bad = true;
+      }
+      const uint32_t real_mask = __ballot_sync(0xFFFFFFFFu, valid && !sent);
+      const uint32_t sent_mask = __ballot_sync(0xFFFFFFFFu, valid && sent);
+      if (seen_sentinel && real_mask) lane_bad = true;
+      if (sent_mask) {
+        const int first_sent = __ffs(sent_mask) - 1;
+        if (real_mask >> first_sent) lane_bad = true;
+      }
+      int left = __shfl_up_sync(0xFFFFFFFFu, loc, 1);
+      if (lane == 0) left = prev_loc;
+      if (valid && !sent && left >= 0 && (lane == 0 || ((real_mask >> (lane - 1)) & 1u)) && loc <= left)
+        lane_bad = true;
+      if (real_mask) prev_loc = __shfl_sync(0xFFFFFFFFu, loc, 31 - __clz(real_mask));
+      seen_sentinel |= sent_mask != 0u;
+      nreal += __popc(real_mask);
+      if (__any_sync(0xFFFFFFFFu, lane_bad)) bad = true;
+    }
+    if ((w1 - w0) - nreal >= 4) bad = true;
+    if (bad && lane == 0) record_status(status, FLASHSPMM_ERR_CORRUPT_FORMAT);
+  }
+}
+
+int enc_grid(int64_t num_tiles) {
+  const int64_t blocks = (num_tiles + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  return static_cast<int>(max64(1, min64(blocks, 148 * 64)));
+}
+
+}  // namespace
+
+cudaError_t launch_tcsl_count(const void* A, int32_t M, int32_t K, int32_t tile_m, int32_t tile_k,
+                              int32_t* tile_offsets, int64_t* nnz, cudaStream_t s) {
+  const int TK = (K + tile_k - 1) / tile_k;
+  const int64_t nt = static_cast<int64_t>((M + tile_m - 1) / tile_m) * TK;
+  if (nt > 0) {
+    tcsl_count_kernel<<<enc_grid(nt), kEncThreads, 0, s>>>(static_cast<const uint4*>(A), M, K, tile_m, tile_k,
+                                                          TK, nt, tile_offsets);
+    note_launch();
+  }
+  tcsl_scan_kernel<<<1, kScanThreads, 0, s>>>(tile_offsets, nt, nnz, device_status_ptr());
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tcsl_fill(const void* A, int32_t M, int32_t K, int32_t tile_m, int32_t tile_k,
+                             const int32_t* tile_offsets, uint32_t* words, int64_t capacity, cudaStream_t s) {
+  const int TK = (K + tile_k - 1) / tile_k;
+  const int64_t nt = static_cast<int64_t>((M + tile_m - 1) / tile_m) * TK;
+  if (nt == 0) return cudaSuccess;
+  tcsl_fill_kernel<<<enc_grid(nt), kEncThreads, 0, s>>>(static_cast<const uint4*>(A), M, K, tile_m, tile_k, TK,
+                                                       nt, tile_offsets, words, capacity, device_status_ptr());
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tcsl_validate(const flashspmm_tcsl* A, cudaStream_t s) {
+  const int TK = (A->K + A->tile_k - 1) / A->tile_k;
+  const int64_t nt = static_cast<int64_t>((A->M + A->tile_m - 1) / A->tile_m) * TK;
+  if (nt == 0) return cudaSuccess;
+  tcsl_validate_kernel<<<enc_grid(nt), kEncThreads, 0, s>>>(A->tile_offsets, A->words, A->nwords, A->M, A->K,
+                                                           A->tile_m, A->tile_k, TK, nt, device_status_ptr());
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace flashspmm
