@@ -52,6 +52,9 @@ extern "C" {
 
 #define FLASHSPMM_ABI_VERSION 1
 
+/* Bytes of the fixed device scratch behind flashspmm_spmm_lscd_noalloc. */
+#define FLASHSPMM_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
 typedef enum {
   FLASHSPMM_OK = 0,
   FLASHSPMM_ERR_INVALID_ARG = 1,    /* null pointer, negative size, mismatched view */
@@ -149,6 +152,27 @@ flashspmm_status flashspmm_spmm_lscd(const flashspmm_tcsl* A, const void* B, voi
 flashspmm_status flashspmm_spmm_lscd_host(const flashspmm_tcsl* A, const void* B_host, void* C_host, void* B_dev,
                                           void* C_dev, int32_t M, int32_t K, int32_t N, int32_t split_k,
                                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* flashspmm_spmm_lscd without a workspace argument.  The paper has no
+ * counterpart to this call; it exists for callers that cannot allocate device
+ * memory on demand, such as a plugin running inside an engine that owns all
+ * device memory and forbids allocation while it executes, or a
+ * latency-critical path that cannot accept cudaMalloc's implicit device
+ * synchronisation.  The call allocates nothing.
+ *   - Its scratch (split-K partial sums and arrival counters) is one
+ *     FLASHSPMM_NOALLOC_SCRATCH_BYTES (16 MiB) array that the library places in
+ *     the memory of every GPU that loads it, held until the process exits.
+ *   - A problem whose flashspmm_spmm_workspace_bytes(M, K, N, split_k) exceeds
+ *     that size returns FLASHSPMM_ERR_CAPACITY and launches nothing (with
+ *     split_k = 0 on a 148-SM B200, every N <= 96 fits).
+ *   - The first call on a device looks up the array's device address; make
+ *     that first call before any stream capture.
+ *   - All calls on a device share the one array and each call clears the
+ *     arrival counters on `stream` before its kernel.  Calls that can overlap
+ *     on the GPU (unordered streams) race on the array and give wrong results.
+ *   - Other arguments and errors as flashspmm_spmm_lscd. */
+flashspmm_status flashspmm_spmm_lscd_noalloc(const flashspmm_tcsl* A, const void* B, void* C, int32_t M, int32_t K,
+                                             int32_t N, int32_t split_k, void* stream);
 
 /* Synchronises `stream`, then reads and clears the library's device status
  * word for the current device: FLASHSPMM_OK or the first error a kernel

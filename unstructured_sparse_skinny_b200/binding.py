@@ -59,6 +59,7 @@ def load_library():
         "flashspmm_spmm_workspace_bytes": (SZ, [I32, I32, I32, I32]),
         "flashspmm_spmm_lscd": (ctypes.c_int, [VP, P, P, I32, I32, I32, I32, P, SZ, P]),
         "flashspmm_spmm_lscd_host": (ctypes.c_int, [VP, P, P, P, P, I32, I32, I32, I32, P, SZ, P]),
+        "flashspmm_spmm_lscd_noalloc": (ctypes.c_int, [VP, P, P, I32, I32, I32, I32, P]),
         "flashspmm_get_device_status": (ctypes.c_int, [P]),
         "flashspmm_launch_count": (ctypes.c_uint64, []),
     }
@@ -198,6 +199,26 @@ def spmm_lscd_host(tcsl_A: TCSL, B_host: torch.Tensor, C_host: torch.Tensor, B_d
                                         workspace.data_ptr() if workspace is not None else None,
                                         workspace.numel() if workspace is not None else 0,
                                         _stream_handle(stream)), "spmm_lscd_host")
+
+
+def spmm_lscd_noalloc(tcsl_A: TCSL, B: torch.Tensor, C: torch.Tensor | None = None, split_k: int = 0,
+                      stream=None) -> torch.Tensor:
+    """C = A x B through the allocation-free entry point (library-held scratch).
+
+    For callers that cannot allocate device memory on demand; see
+    flashspmm_spmm_lscd_noalloc in include/flashspmm.h for the size limit and
+    the rule that overlapping calls on one device must not run concurrently."""
+    lib = load_library()
+    if B.dtype != torch.float16 or B.dim() != 2 or not B.is_cuda or not B.is_contiguous():
+        raise TypeError("B must be a contiguous [N, K] float16 CUDA tensor")
+    N, K = B.shape
+    M = tcsl_A.M
+    if C is None:
+        C = torch.empty((N, M), dtype=torch.float16, device=B.device)
+    v = tcsl_A.view()
+    _check(lib.flashspmm_spmm_lscd_noalloc(ctypes.byref(v), B.data_ptr(), C.data_ptr(), M, K, N, split_k,
+                                           _stream_handle(stream)), "spmm_lscd_noalloc")
+    return C
 
 
 def check_device_status(stream=None) -> None:

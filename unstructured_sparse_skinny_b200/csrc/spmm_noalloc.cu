@@ -1,0 +1,77 @@
+// Allocation-free form of the SpMM entry point.
+//
+// flashspmm_spmm_lscd needs a caller-provided device workspace for its split-K
+// partial sums and arrival counters.  Some callers cannot obtain one on
+// demand: plugins running inside a host engine that owns every byte of device
+// memory and forbids allocation while it executes, or latency-critical paths
+// where cudaMalloc's implicit device synchronisation is not acceptable.  This
+// file gives them flashspmm_spmm_lscd_noalloc, which takes its scratch from a
+// fixed-size array that the library itself places in device memory when it is
+// loaded, so the call allocates nothing.
+#include <atomic>
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace flashspmm {
+namespace {
+
+// Scratch shared by every flashspmm_spmm_lscd_noalloc call on a device.  Each
+// GPU that loads the library holds its own copy until the process exits.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FLASHSPMM_NOALLOC_SCRATCH_BYTES];
+
+// In host code `g_noalloc_scratch` names a host-side stand-in, not device
+// memory; the device address is looked up once per device.
+void* noalloc_scratch_ptr() {
+  static std::atomic<void*> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  void* p = cache[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_noalloc_scratch) != cudaSuccess || a == nullptr) return nullptr;
+    p = a;
+    cache[dev].store(p, std::memory_order_release);
+  }
+  return p;
+}
+
+bool aligned16_ptr(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace flashspmm
+
+using namespace flashspmm;
+
+extern "C" flashspmm_status flashspmm_spmm_lscd_noalloc(const flashspmm_tcsl* A, const void* B, void* C, int32_t M,
+                                                        int32_t K, int32_t N, int32_t split_k, void* stream) {
+  if (!A || M < 0 || K < 0 || N < 0 || A->M != M || A->K != K || A->nwords < 0 || A->nwords > INT32_MAX ||
+      !A->tile_offsets || (A->nwords > 0 && !A->words))
+    return FLASHSPMM_ERR_INVALID_ARG;
+  if (A->tile_m != 64 || A->tile_k != 64 || N > 256 || K % 8 != 0) return FLASHSPMM_ERR_UNSUPPORTED;
+  if (A->words && !aligned16_ptr(A->words)) return FLASHSPMM_ERR_ALIGNMENT;
+  if ((A->nwords & 3) != 0) return FLASHSPMM_ERR_CORRUPT_FORMAT;
+  if (M == 0 || N == 0) return FLASHSPMM_OK;
+  if (!C) return FLASHSPMM_ERR_INVALID_ARG;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev <= 0) return FLASHSPMM_ERR_NO_DEVICE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (K == 0) {
+    return cudaMemsetAsync(C, 0, static_cast<size_t>(M) * N * 2, s) == cudaSuccess ? FLASHSPMM_OK
+                                                                                    : FLASHSPMM_ERR_CUDA;
+  }
+  if (!B) return FLASHSPMM_ERR_INVALID_ARG;
+  if (!aligned16_ptr(B)) return FLASHSPMM_ERR_ALIGNMENT;
+  const int sms = device_sm_count();
+  if (sms <= 0) return FLASHSPMM_ERR_NO_DEVICE;
+  const SpmmPlan plan = make_spmm_plan(M, K, N, split_k, sms);
+  if (plan.workspace_bytes > static_cast<size_t>(FLASHSPMM_NOALLOC_SCRATCH_BYTES)) return FLASHSPMM_ERR_CAPACITY;
+  void* scratch = nullptr;
+  if (plan.workspace_bytes > 0) {
+    scratch = noalloc_scratch_ptr();
+    if (!scratch) return FLASHSPMM_ERR_CUDA;
+  }
+  // The launcher clears the arrival counters on the stream before the kernel;
+  // the partial sums are always written before they are read.
+  return launch_spmm_lscd(A, B, C, M, K, N, plan, scratch, s);
+}
