@@ -171,3 +171,12 @@ def test_workspace_too_small_is_rejected():
     with pytest.raises(fs.FlashSpmmError) as e:
         fs.spmm_lscd(t, torch.from_numpy(B).cuda(), workspace=ws)
     assert e.value.status == 4
+
+
+@pytest.mark.parametrize("s_pct", [95, 99])
+def test_producer_far_ahead_high_sparsity(s_pct):
+    """Large, very sparse problem: the word producer runs many steps ahead of the
+    consumers, so step metadata slots are reused while earlier chunks are still
+    being consumed (a liveness case: must finish without a timeout)."""
+    W, B = _case(9216, 9216, 8, s_pct, key=(212, s_pct))
+    assert_parity(gpu_spmm(gpu_encode(W), B), *_oracle(W, B), f"9216^2 s={s_pct}")

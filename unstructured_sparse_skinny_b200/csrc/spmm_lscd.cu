@@ -55,7 +55,8 @@ constexpr int kGroups = 2;                          // independent decompress gr
 constexpr int kGroupWarps = 4, kGroupThreads = kGroupWarps * 32;
 constexpr int kNumDenseBufs = 4;                    // step n uses dense buffer n % 4 (group n % 2)
 constexpr int kBarEpi = 1, kBarGroup0 = 2;          // named barrier ids (groups use 2..5)
-constexpr int kNumSlots = 64;                       // per-step metadata / barrier slots
+constexpr int kNumSlots = 128;                      // per-step metadata / barrier slots (< 256: 8-bit field)
+constexpr int kBatch = 32;                          // steps published per producer batch (one per lane)
 constexpr int kMinStepsPerPiece = 4;
 static_assert(kWarpDec + kGroups * kGroupWarps == kThreads / 32, "warp roles");
 
@@ -67,7 +68,7 @@ struct Cfg {
   static constexpr int kSlabsPerReq = kBSlabBytes >= 16384 ? 1 : 16384 / kBSlabBytes;  // K tiles per TMA request
   static constexpr int kReqBytes = kSlabsPerReq * kBSlabBytes;
   static constexpr int kNumReq = N_MMA <= 128 ? 3 : 2;   // B requests in flight
-  static constexpr int kRingBytes = 64 * 1024;  // a power of two: positions wrap with a mask
+  static constexpr int kRingBytes = N_MMA <= 128 ? 96 * 1024 : 64 * 1024;
   static constexpr int kRingWords = kRingBytes / 4;
   static constexpr int kChunkTarget = 16 * 1024;  // bytes per published chunk
   static constexpr int kTmemCols = 2 * N_MMA < 32 ? 32 : 2 * N_MMA;
@@ -85,7 +86,6 @@ struct Cfg {
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   // a chunk is at most the target plus one step with two dense tiles
   static_assert(kRingBytes >= kChunkTarget + 2 * kMaxTileWords * 4, "ring must hold the largest chunk");
-  static_assert((kRingBytes & (kRingBytes - 1)) == 0, "ring size must be a power of two");
 };
 
 struct SpmmParams {
@@ -160,30 +160,30 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
-// Thread t of the group takes words t, t + T, t + 2T, ... (T = group size),
-// so each warp-wide store covers 32 consecutive words (a few rows of the
-// tile, few bank conflicts); the next four words are loaded before the
-// current four are stored.
+// Thread t of the group takes words 4t..4t+3, 4(t+T).. (T = group size) with
+// one 16-byte load each (a tile's list and its ring position are multiples of
+// 4 words, so a load never straddles the ring's end); two loads are in flight
+// before the stores.
 template <int RW>
 __device__ __forceinline__ void scatter_range(const uint32_t* ring, uint32_t pos, int cnt, uint32_t base_u32,
                                               int gtid, uint32_t& seen) {
-  constexpr int kU = 4;
-  auto load = [&](int i, uint32_t (&w)[kU]) {
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int k = i + u * kGroupThreads;
-      w[u] = k < cnt ? ring[(pos + static_cast<uint32_t>(k)) & (RW - 1)] : 0xFFFF0000u;
-    }
-  };
-  uint32_t cur[kU];
-  load(gtid, cur);
-  for (int i = gtid; i < cnt; i += kU * kGroupThreads) {
-    uint32_t nxt[kU];
-    load(i + kU * kGroupThreads, nxt);
-#pragma unroll
-    for (int u = 0; u < kU; ++u) scatter_word(base_u32, cur[u], seen);
-#pragma unroll
-    for (int u = 0; u < kU; ++u) cur[u] = nxt[u];
+  const uint4* ring4 = reinterpret_cast<const uint4*>(ring);
+  for (int i = 4 * gtid; i < cnt; i += 8 * kGroupThreads) {
+    const int i2 = i + 4 * kGroupThreads;
+    uint32_t idx = pos + static_cast<uint32_t>(i);
+    if (idx >= static_cast<uint32_t>(RW)) idx -= RW;
+    uint32_t idx2 = pos + static_cast<uint32_t>(i2);
+    if (idx2 >= static_cast<uint32_t>(RW)) idx2 -= RW;
+    const uint4 w = ring4[idx >> 2];
+    const uint4 w2 = i2 < cnt ? ring4[idx2 >> 2] : make_uint4(0xFFFF0000u, 0xFFFF0000u, 0xFFFF0000u, 0xFFFF0000u);
+    scatter_word(base_u32, w.x, seen);
+    scatter_word(base_u32, w.y, seen);
+    scatter_word(base_u32, w.z, seen);
+    scatter_word(base_u32, w.w, seen);
+    scatter_word(base_u32, w2.x, seen);
+    scatter_word(base_u32, w2.y, seen);
+    scatter_word(base_u32, w2.z, seen);
+    scatter_word(base_u32, w2.w, seen);
   }
 }
 
@@ -328,10 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t start_mask = __ballot_sync(0xFFFFFFFFu, start);
       int L0 = 0;
       while (L0 < cnt) {
-        // slots of the steps about to be published must be free
+        // Slots of the steps about to be published must be free.  A step's
+        // barrier is also waited on (by parity) by the consumers of the later
+        // steps of its chunk, so slot s - kNumSlots is reused only once every
+        // step that may share its chunk (chunks never leave a batch, hence
+        // the next kBatch - 1 steps) has been consumed.
         int fail = 0;
         if (lane == 0) {
-          const int64_t need = n + (cnt - L0) - 1 - kNumSlots;
+          const int64_t need = n + (cnt - L0) - 1 - kNumSlots + (kBatch - 1);
           while (!fail && next_confirm <= need) fail = !confirm_next();
         }
         if (__shfl_sync(0xFFFFFFFFu, fail, 0)) { stop = true; break; }
@@ -559,28 +563,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------ decompress (rst_smem + extract)
-    // Group g owns dense buffer g and every kGroups-th step; groups never wait
-    // on one another, so kGroups steps are expanded concurrently.
+    // Group g takes every kGroups-th step and alternates between dense
+    // buffers g and g + 2, so the buffer it zeroes for its next step was last
+    // read by the MMAs of two steps earlier.  Two group barriers per step: one
+    // after the words have landed (which also orders the zero-fill), one
+    // after the scatter.
     const int g = (warp - kWarpDec) / kGroupWarps;
     const int gtid = threadIdx.x - (kWarpDec + g * kGroupWarps) * 32;
     const uint32_t bar_id = kBarGroup0 + g;
     const uint32_t* rw = reinterpret_cast<const uint32_t*>(ring);
     uint32_t seen = 0;
-    int64_t use = 0;
-    for (int64_t q = rg.b + g, n = g; q < rg.e; q += kGroups, n += kGroups, ++use) {
-      const int s = static_cast<int>(n % kNumSlots);
-      const int dbi = static_cast<int>(n % kNumDenseBufs);  // dense buffer of this step
-      const int64_t duse = n / kNumDenseBufs;              // how many times it was used before
-      uint8_t* dbuf = dense + dbi * kDenseBytes;
-      const uint32_t dense_u32 = smem_u32(dbuf);
-      // the group leader waits; the other threads sleep in the named barrier
-      bool ok = true;
-      if (gtid == 0) ok = mbar_wait(&a_empty[dbi], static_cast<uint32_t>((duse & 1) ^ 1), abort_flag, budget, p.status);
-      if (named_barrier_or(bar_id, kGroupThreads, !ok)) break;
-      uint4* dz = reinterpret_cast<uint4*>(dbuf);
+    auto zero_buffer = [&](int dbi) {
+      uint4* dz = reinterpret_cast<uint4*>(dense + dbi * kDenseBytes);
 #pragma unroll
       for (int i = 0; i < kDenseBytes / 16 / kGroupThreads; ++i) dz[i * kGroupThreads + gtid] = make_uint4(0, 0, 0, 0);
-      if (gtid == 0) {
+    };
+    bool next_ok = true;
+    if (rg.b + g < rg.e) zero_buffer(g);  // first use of the buffer: nothing to wait for
+    for (int64_t q = rg.b + g, n = g; q < rg.e; q += kGroups, n += kGroups) {
+      const int s = static_cast<int>(n % kNumSlots);
+      const int dbi = static_cast<int>(n % kNumDenseBufs);
+      const uint32_t dense_u32 = smem_u32(dense + dbi * kDenseBytes);
+      // the group leader waits for the words; the others sleep in the barrier
+      bool ok = next_ok;
+      if (gtid == 0 && ok) {
         ok = mbar_wait(&words_full[s], static_cast<uint32_t>((n / kNumSlots) & 1), abort_flag, budget, p.status);
         if (ok) {
           const int fz = meta[s].z;  // chunk whose copy carries this step's words
@@ -597,6 +603,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (gtid == 0) {
         mbar_arrive(&a_full[dbi]);
         mbar_arrive(&words_empty[s]);
+      }
+      // zero the buffer of this group's next step once its previous MMAs retired
+      const int64_t n2 = n + kGroups;
+      if (q + kGroups < rg.e) {
+        const int d2 = static_cast<int>(n2 % kNumDenseBufs);
+        next_ok = mbar_wait(&a_empty[d2], static_cast<uint32_t>(((n2 / kNumDenseBufs) & 1) ^ 1), abort_flag, budget,
+                            p.status);
+        if (next_ok) zero_buffer(d2);
       }
     }
     if (seen >> 28) record_status(p.status, FLASHSPMM_ERR_CORRUPT_FORMAT);
