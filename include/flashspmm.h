@@ -174,6 +174,13 @@ flashspmm_status flashspmm_spmm_lscd_host(const flashspmm_tcsl* A, const void* B
 flashspmm_status flashspmm_spmm_lscd_noalloc(const flashspmm_tcsl* A, const void* B, void* C, int32_t M, int32_t K,
                                              int32_t N, int32_t split_k, void* stream);
 
+/* Failure-path diagnostic: launches one thread that waits on an mbarrier
+ * nothing completes, bounded by timeout_us (1 .. 1e6) microseconds, exactly as
+ * the SpMM pipeline's waits are bounded.  When the budget runs out the kernel
+ * records FLASHSPMM_ERR_TIMEOUT in the device status word and returns; the
+ * context stays usable.  Returns FLASHSPMM_ERR_INVALID_ARG outside the range. */
+flashspmm_status flashspmm_selftest_wait_timeout(uint32_t timeout_us, void* stream);
+
 /* Synchronises `stream`, then reads and clears the library's device status
  * word for the current device: FLASHSPMM_OK or the first error a kernel
  * recorded since the last read. */

@@ -61,6 +61,7 @@ def load_library():
         "flashspmm_spmm_lscd_host": (ctypes.c_int, [VP, P, P, P, P, I32, I32, I32, I32, P, SZ, P]),
         "flashspmm_spmm_lscd_noalloc": (ctypes.c_int, [VP, P, P, I32, I32, I32, I32, P]),
         "flashspmm_get_device_status": (ctypes.c_int, [P]),
+        "flashspmm_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, P]),
         "flashspmm_launch_count": (ctypes.c_uint64, []),
     }
     for name, (res, args) in sig.items():
