@@ -123,6 +123,13 @@ size_t flashspmm_spmm_workspace_bytes(int32_t M, int32_t K, int32_t N, int32_t s
 
 /* LSCD SpMM [lscd][core-formulas]: C = A x B.
  *   A          Tiled-CSL view with tile_m = tile_k = 64; A->M == M, A->K == K.
+ *              Tile offsets that break the format (negative, unaligned, past
+ *              nwords, a tile longer than 4096 words) record
+ *              FLASHSPMM_ERR_CORRUPT_FORMAT and those tiles are skipped.  Word
+ *              contents are not checked here: a word whose loc lies outside
+ *              the tile (other than the sentinel) is ignored, so the result is
+ *              unspecified but no memory outside the call's buffers is touched;
+ *              flashspmm_tcsl_validate finds such words.
  *   B          device fp16, K x N column-major (a contiguous [N][K] array),
  *              16-byte aligned, K % 8 == 0.  B must be finite: the product is
  *              computed densely per tile, so a non-finite B value meets the

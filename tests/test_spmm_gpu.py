@@ -142,18 +142,22 @@ def test_host_buffer_entry_point_matches_device_path():
     assert C_host.numpy().tobytes() == dev.tobytes()
 
 
-def test_corrupt_words_are_reported_not_faulted():
+def test_corrupt_data_is_contained_and_reported():
+    """A word with an out-of-tile loc is skipped by the SpMM (memory-safe, result
+    unspecified) and reported by the validator; corrupt tile offsets are
+    reported by the SpMM itself."""
     W, B = _case(512, 512, 8, 80, key=(210, 0))
     t = gpu_encode(W)
     w = t.words.clone()
-    w[1] = int(np.uint32(0x3C00 | (5000 << 16)).view(np.int32))  # loc beyond the tile: skipped and flagged
+    w[1] = int(np.uint32(0x3C00 | (5000 << 16)).view(np.int32))  # loc beyond the tile
     bad = fs.TCSL(t.tile_offsets, w, t.nnz, t.M, t.K)
     fs.spmm_lscd(bad, torch.from_numpy(B).cuda())
+    fs.check_device_status()  # the SpMM does not check word contents
     with pytest.raises(fs.FlashSpmmError) as e:
-        fs.check_device_status()
+        fs.tcsl_validate(bad)
     assert e.value.status == 6
     off = t.tile_offsets.clone()
-    off[1] += 1  # misaligned tile start: the copy is skipped and flagged
+    off[1] += 1  # misaligned tile start: the tile is skipped and flagged
     bad = fs.TCSL(off, t.words, t.nnz, t.M, t.K)
     fs.spmm_lscd(bad, torch.from_numpy(B).cuda())
     with pytest.raises(fs.FlashSpmmError) as e:

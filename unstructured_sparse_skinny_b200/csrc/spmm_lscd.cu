@@ -163,25 +163,23 @@ __device__ __forceinline__ uint32_t ldg_word(const uint32_t* ptr, int slot, int 
 // Writes one word's value into a strip's 64 x 64 half of the dense buffer at
 // its swizzled place.  loc = r*64 + c; the unswizzled byte offset is
 // 2*loc = r*128 + 2c, and the 128-byte swizzle XORs the 16-byte chunk index
-// (bits 4-6) with r mod 8 (bits 7-9 of the same offset).  Sentinels are
-// skipped; a corrupt loc >= 4096 stays inside the half (masked) and shows in
-// `hi`: w + 2^16 wraps a sentinel to 0 and exceeds 0x1000FFFF only for a loc
-// in [4096, 0xFFFE] (a max, so the compiler may combine words in any order).
-__device__ __forceinline__ void scatter_word(uint32_t half_u32, uint32_t w, uint32_t& hi) {
-  const uint32_t x = (w >> 15) & 0x1FFEu;
-  const uint32_t off = x ^ ((x >> 3) & 0x70u);
+// (bits 4-6) with r mod 8 (bits 7-9 of the same offset).  Only words with
+// loc < 4096 are written: the sentinel (loc 0xFFFF) and any corrupt loc
+// beyond the tile are skipped by the same test, so no write leaves the half.
+__device__ __forceinline__ void scatter_word(uint32_t half_u32, uint32_t w) {
+  // half_u32 is 1024-aligned, so the swizzle XOR may be applied after adding it
+  const uint32_t addr = (half_u32 + 2u * (w >> 16)) ^ ((w >> 18) & 0x70u);
   asm volatile(
       "{\n\t.reg .pred q;\n\t"
-      "setp.lt.u32 q, %1, 0xFFFF0000;\n\t"
-      "@q st.shared.u16 [%0], %1;\n\t}" ::"r"(half_u32 + off),
+      "setp.lt.u32 q, %1, 0x10000000;\n\t"
+      "@q st.shared.u16 [%0], %1;\n\t}" ::"r"(addr),
       "r"(w));
-  hi = max(hi, w + 0x10000u);
 }
 
 // A load round of a decompress warp: words [base, end) of one strip tile,
 // at most kRoundWords of them.
 struct Round {
-  int64_t k;  // index of the step among the warp's steps
+  int k;      // index of the step among the warp's steps
   bool first, last, valid;
 };
 
@@ -310,10 +308,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t bdesc =
             smem_desc_k_sw128(b_base + static_cast<uint32_t>(r * Cf::kReqBytes + jk * Cf::kBSlabBytes));
         const uint32_t tmem_d = tmem_base + static_cast<uint32_t>(ac * N_MMA);
-        if (leader) {
+        uint64_t ad[kTile / 16], bd[kTile / 16];  // K = 16 per MMA: advance 32 bytes inside the swizzle atom
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk)  // K = 16 per MMA: advance 32 bytes inside the swizzle atom
-            umma_f16_ss(tmem_d, adesc + 2 * kk, bdesc + 2 * kk, Cf::kIdesc, (first && kk == 0) ? 0u : 1u);
+        for (int kk = 0; kk < kTile / 16; ++kk) { ad[kk] = adesc + 2 * kk; bd[kk] = bdesc + 2 * kk; }
+        const uint32_t acc0 = first ? 0u : 1u;
+        if (leader) {
+          umma_f16_ss(tmem_d, ad[0], bd[0], Cf::kIdesc, acc0);
+#pragma unroll
+          for (int kk = 1; kk < kTile / 16; ++kk) umma_f16_ss(tmem_d, ad[kk], bd[kk], Cf::kIdesc, 1u);
           if (jk == kb - 1 || last) umma_commit(&b_empty[r]);  // request fully used
           if (last) umma_commit(&acc_full[ac]);
         }
@@ -436,7 +438,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t piece_steps = rg.e - rg.b;
     const int64_t my_steps = piece_steps > pair ? (piece_steps - pair + kPairs - 1) / kPairs : 0;
     const uint64_t policy = l2_policy_evict_first();
-    uint32_t seen = 0;
     // Tile offsets of 32 consecutive steps of this warp, one step per lane:
     // the current table (validated) and the next one (loads in flight).
     auto load_tab = [&](int64_t k0, int32_t& ta, int32_t& tb) {
@@ -464,13 +465,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     int32_t ca, cb, na, nb;
-    int64_t tab_base = 0, ik = 0;
+    int tab_base = 0, ik = 0;  // steps of this warp: at most a piece's steps, far below 2^31
     uint32_t ipos = 0;
+    const int my_steps32 = static_cast<int>(my_steps);
     load_tab(0, ca, cb);
     load_tab(32, na, nb);
     validate(ca, cb);
     auto issue = [&](uint32_t (&v)[kRoundRegs], Round& rd) {
-      rd.valid = ik < my_steps;
+      rd.valid = ik < my_steps32;
       if (!rd.valid) return;
       if (ik - tab_base == 32) {
         tab_base += 32;
@@ -479,11 +481,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         validate(ca, cb);
         load_tab(tab_base + 32, na, nb);
       }
-      const int li = static_cast<int>(ik - tab_base);
+      const int li = ik - tab_base;
       const uint32_t a0 = static_cast<uint32_t>(__shfl_sync(0xFFFFFFFFu, ca, li));
       const uint32_t a1 = static_cast<uint32_t>(__shfl_sync(0xFFFFFFFFu, cb, li));
       const uint32_t base = a0 + ipos;
-      const int rem = static_cast<int>(min64(static_cast<int64_t>(a1) - base, kRoundWords));
+      const int rem = min(static_cast<int>(a1 - base), kRoundWords);
       rd.k = ik;
       rd.first = ipos == 0;
       rd.last = base + kRoundWords >= a1;
@@ -500,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     // Buffer set k & 1 is free once the MMAs of group k - 2 have retired.
-    auto wait_set = [&](int64_t k) -> bool {  // every lane tests the barrier: no broadcast needed
+    auto wait_set = [&](int k) -> bool {  // every lane tests the barrier: no broadcast needed
       return mbar_wait(&a_empty[k & 1], static_cast<uint32_t>(((k >> 1) & 1) ^ 1), abort_flag, budget, p.status);
     };
     auto process = [&](const uint32_t (&v)[kRoundRegs], const Round& rd) -> bool {
@@ -515,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const uint32_t hb = smem_u32(half);
 #pragma unroll
-      for (int i = 0; i < kRoundRegs; ++i) scatter_word(hb, v[i], seen);
+      for (int i = 0; i < kRoundRegs; ++i) scatter_word(hb, v[i]);
       if (rd.last) {
         fence_proxy_async_smem();
         __syncwarp();
@@ -537,11 +539,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // completes that group's arrival count, once the set is free (so the
     // arrival cannot count towards the set's previous group).
     const int64_t ngroups = (piece_steps + kPairs - 1) / kPairs;
-    if (ok && my_steps < ngroups && wait_set(my_steps)) {
+    if (ok && my_steps < ngroups && wait_set(my_steps32)) {
       __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[my_steps & 1]);
+      if (lane == 0) mbar_arrive(&a_full[my_steps32 & 1]);
     }
-    if (seen > 0x1000FFFFu) record_status(p.status, FLASHSPMM_ERR_CORRUPT_FORMAT);
   }
 
   tc_fence_before_sync();
