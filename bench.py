@@ -73,6 +73,24 @@ def workload_calls(args, rank: int):
     return calls, "opt66b_layer"
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest x over all ranks (device time of the slowest rank); x itself
+    when running alone.  Every rank must call it at the same point."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_rank_step: int, steps: int, max_ms: float, world: int) -> float:
+    """Whole-job GB/s under weak scaling: every rank moves the same bytes per
+    step, and the job takes as long as its slowest rank."""
+    return world * bytes_per_rank_step * steps / (max_ms * 1e-3) / 1e9
+
+
 def algorithmic_bytes(nnz: int, M: int, K: int, N: int, tile: int = 64) -> int:
     tiles = -(-M // tile) * -(-K // tile)
     return 4 * nnz + 4 * (tiles + 1) + 2 * K * N + 2 * M * N
@@ -372,14 +390,10 @@ def main(argv=None):
     per_call_ms = np.array([[ev[k][i].elapsed_time(ev[k][i + 1]) for i in range(len(graphs))]
                             for k in range(args.steps)])
     step_ms = np.array([ev[k][0].elapsed_time(ev[k][-1]) for k in range(args.steps)])
-    total_ms = float(step_ms.sum())
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(float(step_ms.sum()), world, dev)
     bytes_step = sum(w["bytes"] for w in work)
     flops_step = sum(w["flops"] for w in work)
-    value = world * bytes_step * args.steps / (total_ms * 1e-3) / 1e9
+    value = job_throughput(bytes_step, args.steps, total_ms, world)
     tflops = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
     peak, peak_src = measured_peaks()
     kernel_ms = float(per_call_ms.sum())
@@ -419,13 +433,9 @@ def main(argv=None):
                     fs.spmm_lscd_host(w["t"], bh, ch, w["B"], w["C"], split_k=args.split_k, workspace=ws)
             e1.record(stream)
         stream.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         fs.check_device_status(stream)
-        e2e = {"value": world * bytes_step * args.steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e = {"value": job_throughput(bytes_step, args.steps, e2e_ms, world), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
 
     cpu = None
