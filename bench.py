@@ -53,6 +53,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense cuBLAS context timing")
     return ap.parse_args(argv)
 
 
@@ -410,6 +411,39 @@ def main(argv=None):
                        "frac": round(w["bytes"] / (ms * 1e-3) / 1e9 / peak, 4),
                        "TFLOPs_eff": round(w["flops"] / (ms * 1e-3) / 1e12, 2)})
 
+    # ---- context: the same products as dense fp16 GEMMs (cuBLAS through torch),
+    # the comparison the pages report (LSCD vs dense at 70-90 % zeros).  Not part
+    # of the path; timed the same way (graph replay, inputs larger than L2).
+    dense = None
+    if not args.no_dense:
+        dense_us = []
+        for w in work:
+            Wdense = torch.empty((w["M"], w["K"]), dtype=torch.float16, device=dev).normal_(0, 0.02)
+            Bt = w["B"]
+            out = torch.empty((w["N"], w["M"]), dtype=torch.float16, device=dev)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                torch.matmul(Bt, Wdense.t(), out=out)
+                stream.synchronize()
+                with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+                    torch.matmul(Bt, Wdense.t(), out=out)
+                for _ in range(3):
+                    g.replay()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(10):
+                    g.replay()
+                e1.record(stream)
+            stream.synchronize()
+            dense_us.append(e0.elapsed_time(e1) * 100.0)
+            del Wdense, g
+        for d, us in zip(detail, dense_us):
+            d["dense_cublas_us"] = round(us, 2)
+            d["speedup_vs_dense"] = round(us / d["us_median"], 3)
+        dense = {"us_per_step": round(sum(dense_us), 1),
+                 "speedup_vs_dense": round(sum(dense_us) / (total_ms * 1e3 / args.steps), 3),
+                 "note": "torch.matmul fp16 (cuBLAS) on the same shapes with dense random weights; context only"}
+
     # ---- end to end through the host-buffer C-ABI call (pinned B in, C out)
     e2e = None
     if not args.no_e2e:
@@ -474,6 +508,7 @@ def main(argv=None):
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": int(kernels_per_step * args.steps),
+            "dense_context": dense,
             "clocks": clocks,
             "encode": {"GBps": round(enc_bytes / (enc_ms * 1e-3) / 1e9, 1), "ms": round(enc_ms, 3),
                        "bytes": enc_bytes, "note": "once per matrix, outside the timed region; includes the "

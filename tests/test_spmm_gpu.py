@@ -184,3 +184,14 @@ def test_producer_far_ahead_high_sparsity(s_pct):
     being consumed (a liveness case: must finish without a timeout)."""
     W, B = _case(9216, 9216, 8, s_pct, key=(212, s_pct))
     assert_parity(gpu_spmm(gpu_encode(W), B), *_oracle(W, B), f"9216^2 s={s_pct}")
+
+
+@pytest.mark.parametrize("N", [8, 64])
+def test_sparse_matrix_with_dense_tiles(N):
+    """A very sparse matrix (small load rounds) holding one fully dense 64 x 64
+    tile (4096 words: many rounds for one warp) and one dense row segment."""
+    W, B = _case(1024, 1024, N, 95, key=(213, N))
+    g = np.random.default_rng(213)
+    W[128:192, 320:384] = (g.standard_normal((64, 64)) * 0.02).astype(np.float16)
+    W[600, 0:512] = (g.standard_normal(512) * 0.02).astype(np.float16)
+    assert_parity(gpu_spmm(gpu_encode(W), B), *_oracle(W, B), f"dense tiles N={N}")

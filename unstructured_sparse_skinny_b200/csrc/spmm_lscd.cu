@@ -64,8 +64,11 @@ constexpr int kThreads = (kWarpDec + kDecWarps) * 32;
 constexpr int kEpiThreads = 128;
 constexpr int kNumDense = 2 * kPairs;               // two sets of one buffer per pair
 constexpr int kBarEpi = 1;                          // named barrier id of the epilogue warps
-constexpr int kRoundRegs = 32;                      // words per lane per load round
-constexpr int kRoundWords = kRoundRegs * 32;        // 1024 words per warp round
+// Words per lane per load round (a round is 32x that per warp): 32 for most
+// matrices, 16 when a tile averages at most kSmallRoundMaxWords words, where
+// 32-word rounds would be mostly sentinel slots that still cost instructions.
+constexpr int kRoundRegsLarge = 32, kRoundRegsSmall = 16;
+constexpr int kSmallRoundMaxWords = 448;
 constexpr int kMinStepsPerPiece = 4;
 
 
@@ -177,16 +180,18 @@ __device__ __forceinline__ void scatter_word(uint32_t half_u32, uint32_t w) {
 }
 
 // A load round of a decompress warp: words [base, end) of one strip tile,
-// at most kRoundWords of them.
+// at most 32 * RR of them.
 struct Round {
   int k;      // index of the step among the warp's steps
   bool first, last, valid;
 };
 
-template <int N_MMA>
+template <int N_MMA, int RR>
 __global__ void __launch_bounds__(kThreads, 1)
     spmm_lscd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_b, const SpmmParams p) {
   using Cf = Cfg<N_MMA>;
+  constexpr int kRoundRegs = RR;
+  constexpr int kRoundWords = RR * 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* dense = smem + Cf::kOffDense;
@@ -427,8 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------ decompress (gmem2reg + rst_smem + extract)
     // Warp (pair, h) expands strip h of step `pair` of every group, i.e. the
     // steps pair, pair + 4, ... of the piece, into buffer pair of the group's
-    // buffer set.  Its word lists are streamed in rounds of up to 1024 words (32
-    // per lane, consecutive words on consecutive lanes); the loads of the next
+    // buffer set.  Its word lists are streamed in rounds of up to 32 * RR words
+    // (RR per lane, consecutive words on consecutive lanes); the loads of the next
     // round are issued before the current round is expanded, so one round is
     // always in flight.  The first round of a step waits until the MMAs of
     // the buffer's previous step have retired and zeroes the warp's half of
@@ -612,11 +617,15 @@ flashspmm_status launch_bucket(const flashspmm_tcsl* A, const void* B, void* C, 
   if (cudaGetDevice(&dev) != cudaSuccess) return FLASHSPMM_ERR_CUDA;
   const uint64_t bit = uint64_t(1) << (dev & 63);
   if (!(attr_set_mask.load() & bit)) {
-    if (cudaFuncSetAttribute(spmm_lscd_sm100_kernel<N_MMA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cf::kSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(spmm_lscd_sm100_kernel<N_MMA, kRoundRegsLarge>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(spmm_lscd_sm100_kernel<N_MMA, kRoundRegsSmall>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytes) != cudaSuccess)
       return FLASHSPMM_ERR_CUDA;
     attr_set_mask.fetch_or(bit);
   }
+  const int64_t num_tiles = static_cast<int64_t>(plan.TM) * plan.TK;
+  const bool small_rounds = num_tiles > 0 && A->nwords <= static_cast<int64_t>(kSmallRoundMaxWords) * num_tiles;
 
   SpmmParams p{};
   p.tile_offsets = A->tile_offsets;
@@ -635,7 +644,10 @@ flashspmm_status launch_bucket(const flashspmm_tcsl* A, const void* B, void* C, 
   p.status = device_status_ptr();
 
   if (p.counters && cudaMemsetAsync(p.counters, 0, plan.counter_bytes, s) != cudaSuccess) return FLASHSPMM_ERR_CUDA;
-  spmm_lscd_sm100_kernel<N_MMA><<<plan.num_pieces, kThreads, Cf::kSmemBytes, s>>>(tmap, p);
+  if (small_rounds)
+    spmm_lscd_sm100_kernel<N_MMA, kRoundRegsSmall><<<plan.num_pieces, kThreads, Cf::kSmemBytes, s>>>(tmap, p);
+  else
+    spmm_lscd_sm100_kernel<N_MMA, kRoundRegsLarge><<<plan.num_pieces, kThreads, Cf::kSmemBytes, s>>>(tmap, p);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? FLASHSPMM_OK : FLASHSPMM_ERR_CUDA;
 }
