@@ -12,8 +12,9 @@
 //
 //   gmem2reg  -> 8 decompress warps stream their tiles' word lists from HBM
 //                straight into registers (coalesced 32-bit loads, L1
-//                bypassed, L2 evict-first), one 1024-word round always in
-//                flight per warp while the previous round is expanded;
+//                bypassed, L2 evict-first), one round (1024 words, or 512
+//                for very sparse matrices) always in flight per warp while
+//                the previous round is expanded;
 //   rst_smem  -> each warp zeroes its half (64 rows) of a 128 x 64 dense A
 //   + extract    buffer with 16-byte stores and scatters every word's value
 //                to its swizzled position (UMMA K-major 128-byte layout);
