@@ -188,6 +188,23 @@ flashspmm_status flashspmm_spmm_lscd_noalloc(const flashspmm_tcsl* A, const void
  * context stays usable.  Returns FLASHSPMM_ERR_INVALID_ARG outside the range. */
 flashspmm_status flashspmm_selftest_wait_timeout(uint32_t timeout_us, void* stream);
 
+/* Diagnostics of the work partition [code-layout], computed on the host with
+ * the same functions the SpMM kernel uses (no device needed), for num_sms SMs:
+ *   flashspmm_plan_query  info[0..8] = TM, TK, units U, steps T, mode (0 even
+ *                         pieces, 1 split-K per unit), split, pieces, partial
+ *                         slots, workspace bytes; `ranges` (may be NULL, else
+ *                         2 * pieces int64) receives each piece's [begin, end)
+ *                         in steps (step = unit * TK + K tile).  0, or -1 on
+ *                         bad arguments (M, K, N, num_sms > 0, N <= 256).
+ *   flashspmm_plan_owner  mode 0: the piece holding step q, else -1.
+ *   flashspmm_plan_slot   the workspace slot piece pc writes its partial sum
+ *                         of unit u to, -1 when the plan has no partial sums
+ *                         or the arguments are out of range. */
+int flashspmm_plan_query(int32_t M, int32_t K, int32_t N, int32_t split_k, int32_t num_sms, int64_t* info,
+                         int64_t* ranges);
+int64_t flashspmm_plan_owner(int32_t M, int32_t K, int32_t N, int32_t split_k, int32_t num_sms, int64_t q);
+int64_t flashspmm_plan_slot(int32_t M, int32_t K, int32_t N, int32_t split_k, int32_t num_sms, int64_t pc, int64_t u);
+
 /* Synchronises `stream`, then reads and clears the library's device status
  * word for the current device: FLASHSPMM_OK or the first error a kernel
  * recorded since the last read. */

@@ -63,6 +63,9 @@ def load_library():
         "flashspmm_get_device_status": (ctypes.c_int, [P]),
         "flashspmm_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, P]),
         "flashspmm_launch_count": (ctypes.c_uint64, []),
+        "flashspmm_plan_query": (ctypes.c_int, [I32, I32, I32, I32, I32, P, P]),
+        "flashspmm_plan_owner": (ctypes.c_int64, [I32, I32, I32, I32, I32, ctypes.c_int64]),
+        "flashspmm_plan_slot": (ctypes.c_int64, [I32, I32, I32, I32, I32, ctypes.c_int64, ctypes.c_int64]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -137,6 +140,29 @@ def tcsl_validate(A: TCSL, stream=None) -> None:
     v = A.view()
     _check(lib.flashspmm_tcsl_validate(ctypes.byref(v), s), "tcsl_validate")
     _check(lib.flashspmm_get_device_status(s), "tcsl_validate (device)")
+
+
+def plan(M: int, K: int, N: int, split_k: int, num_sms: int) -> dict:
+    """The SpMM work plan for num_sms SMs, computed on the host by the library's
+    own partition code (diagnostics; no device needed)."""
+    lib = load_library()
+    info = (ctypes.c_int64 * 9)()
+    if lib.flashspmm_plan_query(M, K, N, split_k, num_sms, info, None) != 0:
+        raise FlashSpmmError(1, "plan_query")
+    keys = ("TM", "TK", "U", "T", "mode", "split", "num_pieces", "partial_slots", "workspace_bytes")
+    out = dict(zip(keys, (int(v) for v in info)))
+    ranges = (ctypes.c_int64 * (2 * out["num_pieces"]))()
+    lib.flashspmm_plan_query(M, K, N, split_k, num_sms, info, ranges)
+    out["ranges"] = [(int(ranges[2 * i]), int(ranges[2 * i + 1])) for i in range(out["num_pieces"])]
+    return out
+
+
+def plan_owner(M: int, K: int, N: int, split_k: int, num_sms: int, q: int) -> int:
+    return int(load_library().flashspmm_plan_owner(M, K, N, split_k, num_sms, q))
+
+
+def plan_slot(M: int, K: int, N: int, split_k: int, num_sms: int, pc: int, u: int) -> int:
+    return int(load_library().flashspmm_plan_slot(M, K, N, split_k, num_sms, pc, u))
 
 
 def spmm_workspace_bytes(M: int, K: int, N: int, split_k: int = 0) -> int:

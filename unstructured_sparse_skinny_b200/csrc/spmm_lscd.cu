@@ -113,19 +113,19 @@ struct Range {
   int64_t b, e;
 };
 
-__device__ __forceinline__ Range piece_range(const SpmmParams& p, int64_t pc) {
+__host__ __device__ __forceinline__ Range piece_range(const SpmmParams& p, int64_t pc) {
   if (p.mode == 0) return {pc * p.T / p.num_pieces, (pc + 1) * p.T / p.num_pieces};
   const int64_t u = pc / p.split, c = pc - (pc / p.split) * p.split;
   return {u * p.TK + c * p.TK / p.split, u * p.TK + (c + 1) * p.TK / p.split};
 }
 
 // Piece that owns step q in mode 0: the largest pc with floor(pc*T/P) <= q.
-__device__ __forceinline__ int64_t piece_of_step(const SpmmParams& p, int64_t q) {
+__host__ __device__ __forceinline__ int64_t piece_of_step(const SpmmParams& p, int64_t q) {
   return ((q + 1) * p.num_pieces + p.T - 1) / p.T - 1;
 }
 
 // Workspace slot of piece pc's partial sum for unit u.
-__device__ __forceinline__ int64_t partial_slot(const SpmmParams& p, int64_t pc, int64_t u) {
+__host__ __device__ __forceinline__ int64_t partial_slot(const SpmmParams& p, int64_t pc, int64_t u) {
   if (p.mode == 1) return pc;
   return 2 * pc + ((piece_range(p, pc).b / p.TK) != u ? 1 : 0);
 }
@@ -676,7 +676,11 @@ SpmmPlan make_spmm_plan(int32_t M, int32_t K, int32_t N, int32_t split_k, int nu
     pl.split = 0;
     const int64_t want = (pl.T + kMinStepsPerPiece - 1) / kMinStepsPerPiece;
     pl.num_pieces = static_cast<int32_t>(max64(1, min64(want, num_sms > 1 ? num_sms : 1)));
-    pl.partial_slots = pl.num_pieces > 1 ? 2 * static_cast<int64_t>(pl.num_pieces) : 0;
+    // Partial sums exist only if some piece boundary cuts a unit; the kernel
+    // touches the workspace only for such shared units.
+    bool shared = false;
+    for (int64_t pc = 1; pc < pl.num_pieces && !shared; ++pc) shared = (pc * pl.T / pl.num_pieces) % pl.TK != 0;
+    pl.partial_slots = shared ? 2 * static_cast<int64_t>(pl.num_pieces) : 0;
   } else {
     pl.mode = 1;
     pl.split = split_k < pl.TK ? split_k : pl.TK;
@@ -690,6 +694,18 @@ SpmmPlan make_spmm_plan(int32_t M, int32_t K, int32_t N, int32_t split_k, int nu
   return pl;
 }
 
+// The plan fields the kernel's partition helpers read, filled on the host.
+static SpmmParams plan_params(const SpmmPlan& pl) {
+  SpmmParams p{};
+  p.TM = pl.TM; p.TK = pl.TK; p.U = pl.U; p.T = pl.T;
+  p.mode = pl.mode; p.split = pl.split; p.num_pieces = pl.num_pieces;
+  return p;
+}
+
+static bool plan_args_ok(int32_t M, int32_t K, int32_t N, int32_t num_sms) {
+  return M > 0 && K > 0 && N > 0 && N <= 256 && num_sms > 0;
+}
+
 flashspmm_status launch_spmm_lscd(const flashspmm_tcsl* A, const void* B, void* C, int32_t M, int32_t K,
                                   int32_t N, const SpmmPlan& plan, void* workspace, cudaStream_t s) {
   if (N <= 16) return launch_bucket<16>(A, B, C, M, K, N, plan, workspace, s);
@@ -700,3 +716,39 @@ flashspmm_status launch_spmm_lscd(const flashspmm_tcsl* A, const void* B, void* 
 }
 
 }  // namespace flashspmm
+
+using flashspmm::make_spmm_plan;
+
+extern "C" int flashspmm_plan_query(int32_t M, int32_t K, int32_t N, int32_t split_k, int32_t num_sms, int64_t* info,
+                                    int64_t* ranges) {
+  if (!flashspmm::plan_args_ok(M, K, N, num_sms) || !info) return -1;
+  const flashspmm::SpmmPlan pl = make_spmm_plan(M, K, N, split_k, num_sms);
+  const int64_t vals[9] = {pl.TM, pl.TK, pl.U, pl.T, pl.mode, pl.split, pl.num_pieces, pl.partial_slots,
+                           static_cast<int64_t>(pl.workspace_bytes)};
+  for (int i = 0; i < 9; ++i) info[i] = vals[i];
+  if (ranges) {
+    const flashspmm::SpmmParams p = flashspmm::plan_params(pl);
+    for (int64_t pc = 0; pc < pl.num_pieces; ++pc) {
+      const flashspmm::Range r = flashspmm::piece_range(p, pc);
+      ranges[2 * pc] = r.b;
+      ranges[2 * pc + 1] = r.e;
+    }
+  }
+  return 0;
+}
+
+extern "C" int64_t flashspmm_plan_owner(int32_t M, int32_t K, int32_t N, int32_t split_k, int32_t num_sms,
+                                        int64_t q) {
+  if (!flashspmm::plan_args_ok(M, K, N, num_sms)) return -1;
+  const flashspmm::SpmmPlan pl = make_spmm_plan(M, K, N, split_k, num_sms);
+  if (pl.mode != 0 || q < 0 || q >= pl.T) return -1;
+  return flashspmm::piece_of_step(flashspmm::plan_params(pl), q);
+}
+
+extern "C" int64_t flashspmm_plan_slot(int32_t M, int32_t K, int32_t N, int32_t split_k, int32_t num_sms,
+                                       int64_t pc, int64_t u) {
+  if (!flashspmm::plan_args_ok(M, K, N, num_sms)) return -1;
+  const flashspmm::SpmmPlan pl = make_spmm_plan(M, K, N, split_k, num_sms);
+  if (pc < 0 || pc >= pl.num_pieces || u < 0 || u >= pl.U || pl.partial_slots == 0) return -1;
+  return flashspmm::partial_slot(flashspmm::plan_params(pl), pc, u);
+}
