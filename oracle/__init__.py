@@ -64,6 +64,7 @@ def configure(lib):
     lib.ref_tcsl_count.argtypes = [P, I64, I64, I64, I64, P, P]
     lib.ref_tcsl_fill.argtypes = [P, I64, I64, I64, I64, P, P]
     lib.ref_tcsl_decode.argtypes = [P, P, I64, I64, I64, I64, P]
+    lib.ref_tcsl_reorder_banks.argtypes = [P, P, I64, I64, I64]
     lib.ref_spmm.argtypes = [P, P, I64, I64, I64, I64, P, I64, P, P, P, ctypes.c_int]
     lib.ref_spmm_rows.argtypes = [P, P, I64, I64, I64, I64, P, I64, P, I64, P, P]
     lib.ref_dense.argtypes = [P, P, I64, I64, I64, P]
@@ -72,7 +73,8 @@ def configure(lib):
     lib.ref_half_to_double_array.restype = None
     lib.ref_double_to_half_array.argtypes = [P, P, I64]
     lib.ref_double_to_half_array.restype = None
-    for f in ("ref_tcsl_count", "ref_tcsl_fill", "ref_tcsl_decode", "ref_spmm", "ref_spmm_rows"):
+    for f in ("ref_tcsl_count", "ref_tcsl_fill", "ref_tcsl_decode", "ref_tcsl_reorder_banks", "ref_spmm",
+              "ref_spmm_rows"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -114,15 +116,29 @@ def tcsl_count(A, tile_m: int = 64, tile_k: int = 64):
     return off, int(nnz[0])
 
 
-def tcsl_encode(A, tile_m: int = 64, tile_k: int = 64):
-    """Tiled-CSL encoding of A: (tile_offsets int32, words uint32, nnz)."""
+def tcsl_encode(A, tile_m: int = 64, tile_k: int = 64, order: int = 0):
+    """Tiled-CSL encoding of A: (tile_offsets int32, words uint32, nnz).
+
+    order 0: words of a tile in ascending loc (reading R5).  order 1: the
+    bank-balanced word order v2 (64 x 64 tiles only; see ref_tcsl_reorder_banks)."""
     lib = _load()
     A = _bits16(A)
     M, K = A.shape
     off, nnz = tcsl_count(A, tile_m, tile_k)
     words = np.zeros(int(off[-1]), dtype=np.uint32)
     _check(lib.ref_tcsl_fill(_ptr(A), M, K, tile_m, tile_k, _ptr(off), _ptr(words)), "fill")
+    if order == 1:
+        _check(lib.ref_tcsl_reorder_banks(_ptr(off), _ptr(words), len(off) - 1, tile_m, tile_k), "reorder")
+    elif order != 0:
+        raise ValueError("order must be 0 (ascending loc) or 1 (bank-balanced)")
     return off, words, nnz
+
+
+def bank_of_loc(loc):
+    """Shared-memory bank of the value at in-tile loc in the 64 x 64 swizzled dense tile
+    (the quantity the v2 word order balances)."""
+    x = 2 * np.asarray(loc, dtype=np.int64)
+    return ((x ^ ((x >> 3) & 0x70)) >> 2) & 31
 
 
 def tcsl_decode(off, words, M: int, K: int, tile_m: int = 64, tile_k: int = 64) -> np.ndarray:

@@ -34,6 +34,9 @@
  *   R8 B is K x N stored column-major ([N][K]); C is M x N column-major
  *      ([N][M]).
  *   R9 fp32/fp64 -> fp16 rounding is round-to-nearest-even, overflow to Inf.
+ *   R10 word order v2 (optional, 64 x 64 tiles): the page's bank-aware
+ *      reorder restated for the B200 kernel's swizzled dense tile; see
+ *      ref_tcsl_reorder_banks.  Offsets, words and decode are unchanged.
  *
  * Build: gcc -O2 -ffp-contract=off -fno-fast-math -shared -fPIC -pthread.
  */
@@ -156,6 +159,88 @@ int ref_tcsl_fill(const uint16_t* A, int64_t M, int64_t K, int64_t tile_m, int64
         }
     }
     return REF_OK;
+}
+
+/* Word order v2 (bank-balanced), for 64 x 64 tiles only.
+ *
+ * The page's ahead-of-time reordering (section 3, the bank-conflict-aware
+ * reorder of each tile's NonZeros) exists so that a warp's stores of
+ * consecutive words into the dense shared-memory tile hit distinct banks.
+ * Its A100 rule targets a layout that sm_100a does not use; this is the same
+ * idea for the layout the B200 kernel expands into: the value at loc sits at
+ * byte swz(2*loc) of a 64-row x 128-byte tile with the 128-byte swizzle
+ * swz(x) = x ^ ((x >> 3) & 0x70), so its bank is (swz(2*loc) >> 2) & 31.
+ *
+ * Rule: the tile's real words (first in ascending loc, as R5 leaves them) are
+ * placed window by window, a window being 32 consecutive positions from the
+ * tile start (the last one shorter).  At the start of each window the 32
+ * banks are ranked by how many of the tile's words in them are still
+ * unplaced (most first, ties to the lower bank); the window then takes the
+ * next unplaced word (lowest loc) of each bank in that rank order, skipping
+ * banks with none left, and goes round the ranking again while it has room.
+ * Sentinel padding stays at the tile end.  Offsets, the set of words and the
+ * decoded matrix are those of the ascending order. */
+static uint32_t bank_of_loc(uint32_t loc) {
+    uint32_t x = 2u * loc;
+    uint32_t off = x ^ ((x >> 3) & 0x70u);
+    return (off >> 2) & 31u;
+}
+
+int ref_tcsl_reorder_banks(const int32_t* off, uint32_t* words, int64_t num_tiles, int64_t tile_m,
+                           int64_t tile_k) {
+    if (tile_m != 64 || tile_k != 64 || num_tiles < 0) return REF_ERR_ARG;
+    uint32_t (*list)[4096] = malloc(sizeof(uint32_t[32][4096]));
+    uint32_t* out = malloc(sizeof(uint32_t) * 4096);
+    if (!list || !out) { free(list); free(out); return REF_ERR_CAPACITY; }
+    int cnt[32], taken[32];
+    int rc = REF_OK;
+    for (int64_t t = 0; t < num_tiles && rc == REF_OK; ++t) {
+        int64_t b0 = off[t], e0 = off[t + 1];
+        if (e0 - b0 > 4096) { rc = REF_ERR_CORRUPT; break; }
+        for (int b = 0; b < 32; ++b) cnt[b] = taken[b] = 0;
+        int64_t n = 0;
+        for (int64_t w = b0; w < e0; ++w) {
+            uint32_t word = words[w];
+            if (word == SENTINEL) break;
+            uint32_t loc = word >> 16;
+            if (loc >= 4096) { rc = REF_ERR_CORRUPT; break; }
+            uint32_t b = bank_of_loc(loc);
+            list[b][cnt[b]++] = word;
+            ++n;
+        }
+        if (rc != REF_OK) break;
+        int64_t placed = 0;
+        while (placed < n) {
+            int64_t room = n - placed < 32 ? n - placed : 32;
+            int order[32];
+            for (int b = 0; b < 32; ++b) order[b] = b;
+            /* rank banks by unplaced words, most first, ties to the lower bank (insertion sort) */
+            for (int i = 1; i < 32; ++i) {
+                int b = order[i], j = i;
+                while (j > 0) {
+                    int a = order[j - 1];
+                    int ra = cnt[a] - taken[a], rb = cnt[b] - taken[b];
+                    if (ra > rb || (ra == rb && a < b)) break;
+                    order[j] = a;
+                    --j;
+                }
+                order[j] = b;
+            }
+            while (room > 0) {
+                for (int i = 0; i < 32 && room > 0; ++i) {
+                    int b = order[i];
+                    if (taken[b] < cnt[b]) {
+                        out[placed++] = list[b][taken[b]++];
+                        --room;
+                    }
+                }
+            }
+        }
+        for (int64_t i = 0; i < n; ++i) words[b0 + i] = out[i];
+    }
+    free(list);
+    free(out);
+    return rc;
 }
 
 /* Decoder: zero-fill, then write each non-sentinel word's value at its loc.

@@ -10,6 +10,7 @@ import pytest
 
 import oracle
 from tests import test_oracle as pins
+from tests import test_oracle_v2 as pins_v2
 
 SRC = Path(oracle.__file__).resolve().parent / "tcsl_ref.c"
 
@@ -30,6 +31,11 @@ MUTANTS = {
                      "bk[n] = ref_half_to_double(jb->B[k * jb->N + n]);"),
     "decode_row_from_wrong_field": ("int64_t r = loc / tile_k, c = loc % tile_k;\n            int64_t gr",
                                     "int64_t r = loc % tile_k, c = loc / tile_k;\n            int64_t gr"),
+    "v2_ties_to_higher_bank": ("if (ra > rb || (ra == rb && a < b)) break;",
+                               "if (ra > rb || (ra == rb && a > b)) break;"),
+    "v2_fewest_first": ("if (ra > rb || (ra == rb && a < b)) break;", "if (ra < rb || (ra == rb && a < b)) break;"),
+    "v2_unswizzled_bank": ("uint32_t off = x ^ ((x >> 3) & 0x70u);\n    return (off >> 2) & 31u;",
+                           "uint32_t off = x;\n    return (off >> 2) & 31u;"),
     "sentinel_not_skipped_in_spmm": ("if (loc == 0xFFFF) continue;\n                int64_t r = loc / jb->tile_k",
                                      "if (loc == 0xFFFE) continue;\n                int64_t r = loc / jb->tile_k"),
 }
@@ -45,6 +51,8 @@ def _pin_suite():
     yield pins.test_half_to_double_all_patterns
     yield pins.test_double_to_half_matches_numpy
     yield pins.test_permutation_is_exact_product
+    yield lambda: [pins_v2.test_golden_orders(c) for c in pins_v2.GOLDEN["cases"]]
+    yield lambda: pins_v2.test_v2_is_a_reordering_with_the_rule_properties(80, "uniform")
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
