@@ -28,6 +28,10 @@
  *   - words of a tile in ascending loc, padded to a multiple of 4 words with
  *     the sentinel 0xFFFF0000; tile_m * tile_k <= 65535;
  *   - tile_offsets: int32[num_tiles + 1], in words, tile_offsets[0] = 0.
+ *     The SpMM reads them as absolute indices into `words`, so a view whose
+ *     tile_offsets point into a larger matrix's offsets (a run of whole
+ *     strips, with that matrix's words and nwords) is a valid operand: this
+ *     is how a row-split (tensor-parallel) shard is taken without copying.
  *
  * Conventions for every call:
  *   - Array arguments are DEVICE pointers owned by the caller (the only host
@@ -74,7 +78,7 @@ typedef struct {
   int32_t tile_m, tile_k;       /* format tile; the SpMM kernel needs 64 x 64 */
   int64_t nnz;                  /* stored entries excluding padding (informational) */
   int64_t nwords;               /* == tile_offsets[num_tiles] */
-  const int32_t* tile_offsets;  /* device, num_tiles + 1 entries */
+  const int32_t* tile_offsets;  /* device, num_tiles + 1 entries (absolute word indices) */
   const uint32_t* words;        /* device, nwords entries, 16-byte aligned */
 } flashspmm_tcsl;
 
@@ -110,7 +114,7 @@ flashspmm_status flashspmm_tcsl_fill(const void* A, int32_t M, int32_t K, int32_
                                      const int32_t* tile_offsets, uint32_t* words, int64_t words_capacity,
                                      void* stream);
 
-/* Checked mode: verifies a Tiled-CSL view on the GPU (offsets start at 0,
+/* Checked mode: verifies a whole Tiled-CSL matrix on the GPU (offsets start at 0,
  * non-decreasing, multiples of 4, end at nwords, segment <= roundup4(area);
  * each tile holds real words in strictly ascending in-range loc with nonzero
  * value bits, then only exact sentinels).  Any violation records

@@ -195,3 +195,17 @@ def test_sparse_matrix_with_dense_tiles(N):
     W[128:192, 320:384] = (g.standard_normal((64, 64)) * 0.02).astype(np.float16)
     W[600, 0:512] = (g.standard_normal(512) * 0.02).astype(np.float16)
     assert_parity(gpu_spmm(gpu_encode(W), B), *_oracle(W, B), f"dense tiles N={N}")
+
+
+@pytest.mark.parametrize("r0,r1", [(0, 640), (640, 1000), (192, 448), (960, 1000)])
+def test_row_slice_shard(r0, r1):
+    """A row-split shard (a view sharing the full matrix's words) multiplies to
+    the same rows of the product."""
+    W, B = _case(1000, 768, 16, 80, key=(214, 0))
+    t = gpu_encode(W)
+    shard = t.slice_rows(r0, r1)
+    C = fs.spmm_lscd(shard, torch.from_numpy(B).cuda())
+    fs.check_device_status()
+    off, words, _ = oracle.tcsl_encode(W)
+    C64, absC = oracle.spmm_rows(off, words, 1000, 768, B, np.arange(r0, r1))
+    assert_parity(C.cpu().numpy().T, C64, absC, f"rows {r0}:{r1}")

@@ -87,6 +87,9 @@ def _stream_handle(stream) -> int:
     return int(stream)
 
 
+_SENTINEL_I32 = -65536  # 0xFFFF0000 as int32: the padding word
+
+
 @dataclass
 class TCSL:
     """A Tiled-CSL matrix resident in device memory."""
@@ -105,6 +108,22 @@ class TCSL:
     def view(self) -> _TcslView:
         return _TcslView(self.M, self.K, self.tile_m, self.tile_k, self.nnz, self.nwords,
                          self.tile_offsets.data_ptr(), self.words.data_ptr() if self.nwords else None)
+
+    def slice_rows(self, row_begin: int, row_end: int) -> "TCSL":
+        """Rows [row_begin, row_end) as a Tiled-CSL view for row-split (tensor-parallel)
+        sharding; nothing is copied.  row_begin must start a strip (a multiple of
+        tile_m) and row_end must end one or be M.  The view keeps this matrix's
+        word array: tile offsets are absolute word indices, so the shard's offsets
+        are a slice of the full offsets and every tile finds its words unchanged."""
+        if not (0 <= row_begin < row_end <= self.M) or row_begin % self.tile_m or \
+                (row_end % self.tile_m and row_end != self.M):
+            raise ValueError("a row slice must start and end on strip boundaries")
+        TK = -(-self.K // self.tile_k)
+        i0, i1 = row_begin // self.tile_m, -(-row_end // self.tile_m)
+        offs = self.tile_offsets[i0 * TK:i1 * TK + 1]
+        a, b = (int(x) for x in offs[[0, -1]].tolist())
+        nnz = int((self.words[a:b] != _SENTINEL_I32).sum()) if b > a else 0
+        return TCSL(offs, self.words, nnz, row_end - row_begin, self.K, self.tile_m, self.tile_k)
 
 
 def tcsl_encode(A_dense: torch.Tensor, tile_m: int = 64, tile_k: int = 64, stream=None) -> TCSL:
