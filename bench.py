@@ -47,6 +47,9 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="lscd", choices=["lscd", "reference"])
+    ap.add_argument("--workload", default="opt66b_layer",
+                    choices=[w.name for w in synth.WORKLOADS.values()],
+                    help="named workload (the default is the one the metric is quoted on)")
     ap.add_argument("--case", default=None,
                     help="single SpMM 'M,K,N,sparsity_pct[,structure]' instead of the layer workload")
     ap.add_argument("--split-k", type=int, default=0)
@@ -66,12 +69,17 @@ def workload_calls(args, rank: int):
         M, K, N, s = (int(x) for x in parts[:4])
         st = parts[4] if len(parts) > 4 else "uniform"
         return [(f"case_{M}x{K}", M, K, N, s, st, (90, rank))], f"case {M}x{K} N={N} {s}% {st}"
-    wl = synth.WORKLOADS[2]
+    wl = next(w for w in synth.WORKLOADS.values() if w.name == args.workload)
+    one_mask = len(wl.sparsities) == 1 and len(wl.structures) == 1
     calls = []
-    for n in wl.Ns:
-        for li, mm in enumerate(wl.matmuls):
-            calls.append((mm.name, mm.M, mm.K, n, wl.sparsities[0], wl.structures[0], (2, li + 1000 * rank)))
-    return calls, "opt66b_layer"
+    for s in wl.sparsities:
+        for st in wl.structures:
+            for n in wl.Ns:
+                for li, mm in enumerate(wl.matmuls):
+                    # one matrix per (matmul, sparsity, structure), shared by its N values
+                    name = mm.name if one_mask else f"{mm.name}_{s}pct_{st}"
+                    calls.append((name, mm.M, mm.K, n, s, st, (wl.cfg, li + 1000 * rank)))
+    return calls, wl.name
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
@@ -161,6 +169,20 @@ class ClockSampler:
         pw = [num(f[3]) for f in window if num(f[3]) is not None]
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(window), "power_w_max": max(pw) if pw else None}
+
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def l2_note(work) -> str:
+    """Whether the timed calls can find their weights in L2 (126 MB on B200)."""
+    step_words = sum(w["t"].nwords for w in work) * 4
+    per_n = step_words / len({w["N"] for w in work})
+    if per_n > 2 * L2_BYTES:
+        return (f"inputs larger than L2: every step streams all weight matrices ({per_n / 1e6:.0f} MB of words "
+                "per N), so no matrix is L2-resident when re-read")
+    return (f"inputs smaller than L2 ({per_n / 1e6:.1f} MB of words per N): figures are L2-warm, "
+            "not an HBM measurement")
 
 
 def kernel_source_hash() -> str:
@@ -507,9 +529,7 @@ def main(argv=None):
             "config": {"workload": cfg_name, "tile": "64x64", "Ns": sorted({w['N'] for w in work}),
                        "sparsity_pct": sorted({c[4] for c in calls}), "split_k": args.split_k,
                        "calls_per_step": len(work),
-                       "l2": "inputs larger than L2: every step streams all weight matrices "
-                             f"({sum(w['t'].nwords for w in work) * 4 / len({w['N'] for w in work}) / 1e6:.0f} MB "
-                             "of words per N), so no matrix is L2-resident when re-read",
+                       "l2": l2_note(work),
                        "launch": "one CUDA graph per call, replayed back to back"},
             "effective_tflops": round(tflops, 3),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
