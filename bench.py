@@ -300,6 +300,39 @@ def run_reference(args, calls, cfg_name, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def bench_line(*, world, args, cfg_name, work, calls, value, total_ms, tflops, achieved, peak, peak_src,
+               bytes_step, cpu, e2e, kernels_per_step, dense, clocks, enc_bytes, enc_ms, detail) -> dict:
+    """The one JSON line the benchmark prints (rank 0)."""
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
+        "data": "synthetic",
+        "config": {"workload": cfg_name, "tile": "64x64", "Ns": sorted({w['N'] for w in work}),
+                   "sparsity_pct": sorted({c[4] for c in calls}), "split_k": args.split_k,
+                   "calls_per_step": len(work),
+                   "l2": l2_note(work),
+                   "launch": "one CUDA graph per call, replayed back to back"},
+        "effective_tflops": round(tflops, 3),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic(cfg_name),
+                     "traffic_unit": "DRAM bytes per step (all calls of the step; ncu)",
+                     "algorithmic_bytes_per_step": bytes_step,
+                     "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)" if peak_src == "measured"
+                     else "fallback 6.65 TB/s"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(kernels_per_step * args.steps),
+        "dense_context": dense,
+        "clocks": clocks,
+        "encode": {"GBps": round(enc_bytes / (enc_ms * 1e-3) / 1e9, 1) if enc_ms > 0 else None,
+                   "ms": round(enc_ms, 3), "bytes": enc_bytes,
+                   "note": "once per matrix, outside the timed region; includes the "
+                           "host read of the word count between the two passes"},
+        "detail": detail,
+    }
+
+
 # ---------------------------------------------------------------- GPU leg
 
 def main(argv=None):
@@ -521,33 +554,10 @@ def main(argv=None):
             cpu.pop("seconds", None)
 
     if rank == 0:
-        line = {
-            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
-            "data": "synthetic",
-            "config": {"workload": cfg_name, "tile": "64x64", "Ns": sorted({w['N'] for w in work}),
-                       "sparsity_pct": sorted({c[4] for c in calls}), "split_k": args.split_k,
-                       "calls_per_step": len(work),
-                       "l2": l2_note(work),
-                       "launch": "one CUDA graph per call, replayed back to back"},
-            "effective_tflops": round(tflops, 3),
-            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": profiled_traffic(cfg_name),
-                         "traffic_unit": "DRAM bytes per step (all calls of the step; ncu)",
-                         "algorithmic_bytes_per_step": bytes_step,
-                         "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)" if peak_src == "measured"
-                         else "fallback 6.65 TB/s"},
-            "cpu_baseline": cpu,
-            "e2e": e2e,
-            "gpu_launches": int(kernels_per_step * args.steps),
-            "dense_context": dense,
-            "clocks": clocks,
-            "encode": {"GBps": round(enc_bytes / (enc_ms * 1e-3) / 1e9, 1), "ms": round(enc_ms, 3),
-                       "bytes": enc_bytes, "note": "once per matrix, outside the timed region; includes the "
-                                                   "host read of the word count between the two passes"},
-            "detail": detail,
-        }
+        line = bench_line(world=world, args=args, cfg_name=cfg_name, work=work, calls=calls, value=value,
+                          total_ms=total_ms, tflops=tflops, achieved=achieved, peak=peak, peak_src=peak_src,
+                          bytes_step=bytes_step, cpu=cpu, e2e=e2e, kernels_per_step=kernels_per_step,
+                          dense=dense, clocks=clocks, enc_bytes=enc_bytes, enc_ms=enc_ms, detail=detail)
         print(json.dumps(line), flush=True)
     graphs.clear()
     if world > 1:
