@@ -148,7 +148,13 @@ size_t flashspmm_spmm_workspace_bytes(int32_t M, int32_t K, int32_t N, int32_t s
  *              Results are deterministic for a given (problem, split_k, device).
  *   workspace  device, >= flashspmm_spmm_workspace_bytes(...), 16-byte aligned;
  *              may be NULL when that size is 0.  Holds fp32 partial sums and
- *              per-unit arrival counters; it is cleared by the call itself.
+ *              per-unit arrival counters; the call clears the counters on
+ *              `stream` before its kernel, so the contents need no
+ *              preparation.  Calls that may run concurrently need separate
+ *              workspaces.
+ * The kernel is launched with programmatic stream serialisation: its
+ * prologue may overlap the tail of the previous kernel in the stream, and it
+ * reads no input before that kernel has completed.
  * K == 0 writes zeros to C; M == 0 or N == 0 does nothing. */
 flashspmm_status flashspmm_spmm_lscd(const flashspmm_tcsl* A, const void* B, void* C, int32_t M, int32_t K,
                                      int32_t N, int32_t split_k, void* workspace, size_t workspace_bytes,
@@ -179,8 +185,9 @@ flashspmm_status flashspmm_spmm_lscd_host(const flashspmm_tcsl* A, const void* B
  *   - The first call on a device looks up the array's device address; make
  *     that first call before any stream capture.
  *   - All calls on a device share the one array and each call clears the
- *     arrival counters on `stream` before its kernel.  Calls that can overlap
- *     on the GPU (unordered streams) race on the array and give wrong results.
+ *     arrival counters on `stream` before its kernel.
+ *     Calls that can overlap on the GPU (unordered streams) race on the array
+ *     and give wrong results.
  *   - Other arguments and errors as flashspmm_spmm_lscd. */
 flashspmm_status flashspmm_spmm_lscd_noalloc(const flashspmm_tcsl* A, const void* B, void* C, int32_t M, int32_t K,
                                              int32_t N, int32_t split_k, void* stream);

@@ -71,7 +71,8 @@ extern "C" flashspmm_status flashspmm_spmm_lscd_noalloc(const flashspmm_tcsl* A,
     scratch = noalloc_scratch_ptr();
     if (!scratch) return FLASHSPMM_ERR_CUDA;
   }
-  // The launcher clears the arrival counters on the stream before the kernel;
-  // the partial sums are always written before they are read.
+  // The array keeps whatever the last call left in it.  The launcher clears
+  // the arrival counters (which must start at zero) on the stream before the
+  // kernel; the partial sums are always written before they are read.
   return launch_spmm_lscd(A, B, C, M, K, N, plan, scratch, s);
 }
