@@ -25,8 +25,9 @@
  *     (t = i * ceil(K/tile_k) + j); edge tiles may be ragged;
  *   - loc = r * tile_k + c inside the tile (row-major, full tile_k pitch);
  *   - word = fp16 bits | (loc << 16); stored iff the fp16 bits are not 0x0000;
- *   - words of a tile in ascending loc, padded to a multiple of 4 words with
- *     the sentinel 0xFFFF0000; tile_m * tile_k <= 65535;
+ *   - words of a tile in ascending loc (or, after flashspmm_tcsl_reorder_banks,
+ *     the bank-balanced order; the SpMM accepts either), padded to a multiple
+ *     of 4 words with the sentinel 0xFFFF0000; tile_m * tile_k <= 65535;
  *   - tile_offsets: int32[num_tiles + 1], in words, tile_offsets[0] = 0.
  *     The SpMM reads them as absolute indices into `words`, so a view whose
  *     tile_offsets point into a larger matrix's offsets (a run of whole
@@ -114,11 +115,33 @@ flashspmm_status flashspmm_tcsl_fill(const void* A, int32_t M, int32_t K, int32_
                                      const int32_t* tile_offsets, uint32_t* words, int64_t words_capacity,
                                      void* stream);
 
+/* Optional encoder pass [tiled-csl] (page's ahead-of-time reordering of each
+ * tile's nonzeros, restated for this library's dense tile): rewrites, in
+ * place, the words of every 64 x 64 tile of an ascending-loc encoding into
+ * the bank-balanced order ("word order v2").  The value at loc lands in the
+ * SpMM's shared-memory tile at byte x = 2*loc swizzled as x ^ ((x >> 3) & 0x70),
+ * i.e. in bank (that offset >> 2) & 31.  A tile's real words (those before its
+ * first sentinel) are placed window by window, a window being 32 consecutive
+ * positions from the tile start: at each window's start the banks are ranked
+ * by unplaced words (most first, ties to the lower bank) and the window takes
+ * the lowest-loc unplaced word of each bank in rank order, round after round,
+ * until it is full.  Offsets, the set of words, padding and the decoded
+ * matrix are unchanged; a 32-word store of the SpMM then hits as many
+ * distinct banks as possible.
+ *   tile_offsets  device int32[num_tiles + 1] of an M x K matrix, 64 x 64 tiles.
+ *   words         device uint32[nwords], rewritten in place, 16-byte aligned.
+ * A tile longer than 4096 words or holding a real word with loc >= 4096
+ * records FLASHSPMM_ERR_CORRUPT_FORMAT and is left unchanged.  Tiles other
+ * than 64 x 64 return FLASHSPMM_ERR_UNSUPPORTED. */
+flashspmm_status flashspmm_tcsl_reorder_banks(const int32_t* tile_offsets, uint32_t* words, int64_t nwords, int32_t M,
+                                              int32_t K, int32_t tile_m, int32_t tile_k, void* stream);
+
 /* Checked mode: verifies a whole Tiled-CSL matrix on the GPU (offsets start at 0,
  * non-decreasing, multiples of 4, end at nwords, segment <= roundup4(area);
- * each tile holds real words in strictly ascending in-range loc with nonzero
- * value bits, then only exact sentinels).  Any violation records
- * FLASHSPMM_ERR_CORRUPT_FORMAT in the device status word. */
+ * each tile holds real words with distinct in-range locs and nonzero value
+ * bits, in any order (ascending or bank-balanced), then fewer than four exact
+ * sentinels).  Any violation records FLASHSPMM_ERR_CORRUPT_FORMAT in the
+ * device status word. */
 flashspmm_status flashspmm_tcsl_validate(const flashspmm_tcsl* A, void* stream);
 
 /* Bytes of workspace flashspmm_spmm_lscd needs on the CURRENT device for this

@@ -69,16 +69,67 @@ def test_validate_accepts_and_rejects():
     corruptions = []
     w = words.clone(); w[5] = int(np.int32(np.uint32(0x3C00 | (4096 << 16)).view(np.int32)))  # loc out of tile
     corruptions.append(("loc", t.tile_offsets, w))
-    w = words.clone(); w[0], w[1] = words[1].item(), words[0].item()  # order broken
-    corruptions.append(("order", t.tile_offsets, w))
+    w = words.clone(); w[1] = words[0].item()  # one location stored twice in a tile
+    corruptions.append(("duplicate", t.tile_offsets, w))
     off = t.tile_offsets.clone(); off[3] += 2  # offset not a multiple of 4
     corruptions.append(("offset", off, words))
-    end = int(t.tile_offsets[1].item())
-    w = words.clone(); w[end - 1] = 0x3C00  # value bits nonzero with loc 0 where a sentinel / ascending word was
-    corruptions.append(("tail", t.tile_offsets, w))
+    w = words.clone(); w[5] = int(np.uint32(0xFFFF3C00).view(np.int32))  # sentinel location with value bits
+    corruptions.append(("sentinel", t.tile_offsets, w))
+    w = words.clone(); w[5] = int(words[5].item()) & ~0xFFFF  # a real word whose value bits are zero
+    corruptions.append(("zero value", t.tile_offsets, w))
     for name, o, w in corruptions:
         bad = fs.TCSL(o, w, t.nnz, t.M, t.K)
         with pytest.raises(fs.FlashSpmmError) as e:
             fs.tcsl_validate(bad)
         assert e.value.status == 6, name
     fs.tcsl_validate(t)  # status word was cleared by the failing reads
+
+
+# ---- word order v2 (bank-balanced), the page's ahead-of-time reorder restated for the B200 tile
+
+def _v2_bit_exact(W):
+    t = fs.tcsl_encode(torch.from_numpy(np.ascontiguousarray(W)).cuda(), order=1)
+    fs.check_device_status()
+    off, words, nnz = oracle.tcsl_encode(W, order=1)
+    assert np.array_equal(t.tile_offsets.cpu().numpy(), off)
+    gw = t.words.cpu().numpy().view(np.uint32)
+    assert gw.size == words.size and gw.tobytes() == words.tobytes()
+    assert t.nnz == nnz and t.order == 1
+    return t
+
+
+V2_CASES = [(st, s) for st in ("uniform", "row_magnitude", "power_law", "column_clustered")
+            for s in (0, 50, 70, 80, 90, 99)
+            if not (st == "power_law" and not 40 <= s <= 98)]  # power-law row densities lie in [2 %, 60 %]
+
+
+@pytest.mark.parametrize("structure,s_pct", V2_CASES)
+def test_v2_structures_bit_exact(structure, s_pct):
+    W = synth.sparse_weight(768, 1024, s_pct, structure, (101, s_pct))
+    _v2_bit_exact(W)
+
+
+@pytest.mark.parametrize("M,K", [(200, 136), (130, 72), (1, 8), (64, 64), (2048, 8), (8, 4096), (333, 1000)])
+def test_v2_ragged(M, K):
+    g = np.random.default_rng(M * 7 + K)
+    W = (g.standard_normal((M, K)) * 0.02).astype(np.float16)
+    W[g.random((M, K)) < 0.75] = 0
+    _v2_bit_exact(W)
+
+
+def test_v2_edge_tiles():
+    _v2_bit_exact(np.zeros((128, 192), dtype=np.float16))          # empty tiles
+    _v2_bit_exact(np.ones((128, 128), dtype=np.float16))           # 4096-word tiles, one bank order
+    W = np.zeros((128, 128), dtype=np.float16)
+    W[:, 0] = 1                                                   # every word in the same two banks
+    W[5, 7] = 2
+    _v2_bit_exact(W)
+
+
+def test_v2_validates_and_keeps_decode():
+    W = synth.sparse_weight(1024, 1024, 80, "power_law", (102, 0))
+    t = _v2_bit_exact(W)
+    fs.tcsl_validate(t)
+    off = t.tile_offsets.cpu().numpy()
+    assert np.array_equal(oracle.tcsl_decode(off, t.words.cpu().numpy().view(np.uint32), 1024, 1024),
+                          W.view(np.uint16))

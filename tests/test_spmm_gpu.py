@@ -209,3 +209,15 @@ def test_row_slice_shard(r0, r1):
     off, words, _ = oracle.tcsl_encode(W)
     C64, absC = oracle.spmm_rows(off, words, 1000, 768, B, np.arange(r0, r1))
     assert_parity(C.cpu().numpy().T, C64, absC, f"rows {r0}:{r1}")
+
+
+@pytest.mark.parametrize("structure,s_pct,N", [("uniform", 80, 8), ("uniform", 70, 32), ("power_law", 90, 16),
+                                               ("column_clustered", 80, 64), ("row_magnitude", 50, 128),
+                                               ("uniform", 95, 256)])
+def test_bank_balanced_word_order(structure, s_pct, N):
+    """The SpMM reads either word order: bank-balanced (v2) words give a product
+    within the same bound (the scatter does not depend on the order)."""
+    W, B = _case(2048, 1536, N, s_pct, structure, key=(210, s_pct))
+    t = fs.tcsl_encode(torch.from_numpy(W).cuda(), order=1)
+    fs.check_device_status()
+    assert_parity(gpu_spmm(t, B), *_oracle(W, B), f"v2 {structure} {s_pct}% N={N}")

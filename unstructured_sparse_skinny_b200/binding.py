@@ -56,6 +56,7 @@ def load_library():
         "flashspmm_tcsl_count": (ctypes.c_int, [P, I32, I32, I32, I32, P, P, P]),
         "flashspmm_tcsl_fill": (ctypes.c_int, [P, I32, I32, I32, I32, P, P, I64, P]),
         "flashspmm_tcsl_validate": (ctypes.c_int, [VP, P]),
+        "flashspmm_tcsl_reorder_banks": (ctypes.c_int, [P, P, I64, I32, I32, I32, I32, P]),
         "flashspmm_spmm_workspace_bytes": (SZ, [I32, I32, I32, I32]),
         "flashspmm_spmm_lscd": (ctypes.c_int, [VP, P, P, I32, I32, I32, I32, P, SZ, P]),
         "flashspmm_spmm_lscd_host": (ctypes.c_int, [VP, P, P, P, P, I32, I32, I32, I32, P, SZ, P]),
@@ -100,6 +101,7 @@ class TCSL:
     K: int
     tile_m: int = 64
     tile_k: int = 64
+    order: int = 0              # 0: ascending loc in a tile; 1: bank-balanced (word order v2)
 
     @property
     def nwords(self) -> int:
@@ -123,14 +125,17 @@ class TCSL:
         offs = self.tile_offsets[i0 * TK:i1 * TK + 1]
         a, b = (int(x) for x in offs[[0, -1]].tolist())
         nnz = int((self.words[a:b] != _SENTINEL_I32).sum()) if b > a else 0
-        return TCSL(offs, self.words, nnz, row_end - row_begin, self.K, self.tile_m, self.tile_k)
+        return TCSL(offs, self.words, nnz, row_end - row_begin, self.K, self.tile_m, self.tile_k, self.order)
 
 
-def tcsl_encode(A_dense: torch.Tensor, tile_m: int = 64, tile_k: int = 64, stream=None) -> TCSL:
+def tcsl_encode(A_dense: torch.Tensor, tile_m: int = 64, tile_k: int = 64, stream=None, order: int = 0) -> TCSL:
     """Encode a row-major fp16 ``[M, K]`` device tensor into Tiled-CSL on the GPU.
 
     Runs the count pass, reads the word total back (one host sync), allocates
-    the words with torch, then runs the fill pass."""
+    the words with torch, then runs the fill pass; ``order=1`` adds the
+    in-place bank-balanced reordering (64 x 64 tiles only)."""
+    if order not in (0, 1):
+        raise ValueError("order must be 0 (ascending loc) or 1 (bank-balanced)")
     lib = load_library()
     if A_dense.dtype != torch.float16 or A_dense.dim() != 2 or not A_dense.is_cuda:
         raise TypeError("A_dense must be a 2-D float16 CUDA tensor")
@@ -149,7 +154,10 @@ def tcsl_encode(A_dense: torch.Tensor, tile_m: int = 64, tile_k: int = 64, strea
     words = torch.empty(max(nwords, 0), dtype=torch.int32, device=A.device)
     _check(lib.flashspmm_tcsl_fill(A.data_ptr() if A.numel() else None, M, K, tile_m, tile_k, off.data_ptr(),
                                    words.data_ptr() if nwords else None, nwords, s), "tcsl_fill")
-    return TCSL(off, words, int(nnz.item()), M, K, tile_m, tile_k)
+    if order == 1:
+        _check(lib.flashspmm_tcsl_reorder_banks(off.data_ptr(), words.data_ptr() if nwords else None, nwords, M, K,
+                                                tile_m, tile_k, s), "tcsl_reorder_banks")
+    return TCSL(off, words, int(nnz.item()), M, K, tile_m, tile_k, order)
 
 
 def tcsl_validate(A: TCSL, stream=None) -> None:

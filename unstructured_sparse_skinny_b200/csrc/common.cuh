@@ -25,6 +25,8 @@ cudaError_t launch_tcsl_count(const void* A, int32_t M, int32_t K, int32_t tile_
                               int32_t* tile_offsets, int64_t* nnz, cudaStream_t s);
 cudaError_t launch_tcsl_fill(const void* A, int32_t M, int32_t K, int32_t tile_m, int32_t tile_k,
                              const int32_t* tile_offsets, uint32_t* words, int64_t capacity, cudaStream_t s);
+cudaError_t launch_tcsl_reorder_banks(const int32_t* tile_offsets, uint32_t* words, int64_t num_tiles, int64_t nwords,
+                                      cudaStream_t s);
 cudaError_t launch_tcsl_validate(const flashspmm_tcsl* A, cudaStream_t s);
 
 // Work plan of one SpMM call: how the step space is cut into pieces and how

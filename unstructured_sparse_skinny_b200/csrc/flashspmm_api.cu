@@ -115,6 +115,20 @@ flashspmm_status flashspmm_tcsl_fill(const void* A, int32_t M, int32_t K, int32_
              : FLASHSPMM_ERR_CUDA;
 }
 
+flashspmm_status flashspmm_tcsl_reorder_banks(const int32_t* tile_offsets, uint32_t* words, int64_t nwords, int32_t M,
+                                               int32_t K, int32_t tile_m, int32_t tile_k, void* stream) {
+  if (M < 0 || K < 0 || tile_m <= 0 || tile_k <= 0 || nwords < 0 || nwords > INT32_MAX || !tile_offsets ||
+      (nwords > 0 && !words))
+    return FLASHSPMM_ERR_INVALID_ARG;
+  if (tile_m != 64 || tile_k != 64) return FLASHSPMM_ERR_UNSUPPORTED;
+  if (words && !aligned16(words)) return FLASHSPMM_ERR_ALIGNMENT;
+  if (!have_device()) return FLASHSPMM_ERR_NO_DEVICE;
+  const int64_t nt = static_cast<int64_t>((M + 63) / 64) * ((K + 63) / 64);
+  return launch_tcsl_reorder_banks(tile_offsets, words, nt, nwords, as_stream(stream)) == cudaSuccess
+             ? FLASHSPMM_OK
+             : FLASHSPMM_ERR_CUDA;
+}
+
 flashspmm_status flashspmm_tcsl_validate(const flashspmm_tcsl* A, void* stream) {
   flashspmm_status st = check_view(A);
   if (st != FLASHSPMM_OK) return st;

@@ -8,8 +8,9 @@
 //   1. count:    one warp per tile counts nonzero fp16 bit patterns;
 //   2. scan:     one CTA turns counts into padded running offsets and sums nnz;
 //   3. fill:     one warp per tile compacts the tile in loc order with a warp
-//                prefix sum (no atomics, so positions are deterministic).
-// A fourth kernel validates a given encoding (checked mode).
+//                prefix sum (no atomics, so positions are deterministic);
+//   4. optional: the bank-balanced word order (v2), in place.
+// A further kernel validates a given encoding (checked mode).
 #include "common.cuh"
 #include "sm100_primitives.cuh"
 
@@ -175,17 +176,24 @@ __global__ void __launch_bounds__(kEncThreads) tcsl_fill_kernel(const uint4* __r
   }
 }
 
-// Checked mode: one warp per tile verifies the offsets and the words.
-__global__ void __launch_bounds__(kEncThreads) tcsl_validate_kernel(const int32_t* __restrict__ off,
-                                                                   const uint32_t* __restrict__ words,
-                                                                   int64_t nwords, int M, int K, int tile_m,
-                                                                   int tile_k, int TK, int64_t num_tiles, int* status) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kEncThreads + threadIdx.x) >> 5;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarpsPerBlock;
+// Checked mode: one warp per tile verifies the offsets and the words.  A
+// tile's real words must hold distinct in-range locations with nonzero value
+// bits (in any order, so both the ascending and the bank-balanced word order
+// pass), followed only by exact sentinels, fewer than four of them.
+constexpr int kValWarps = 4;
+constexpr int kValBitmapWords = 65536 / 32;  // one bit per location of the largest tile
+
+__global__ void __launch_bounds__(kValWarps * 32) tcsl_validate_kernel(const int32_t* __restrict__ off,
+                                                                      const uint32_t* __restrict__ words,
+                                                                      int64_t nwords, int M, int K, int tile_m,
+                                                                      int tile_k, int TK, int64_t num_tiles, int* status) {
+  __shared__ uint32_t s_seen[kValWarps][kValBitmapWords];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* seen = s_seen[warp];
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * kValWarps;
   const int area = tile_m * tile_k;
   const int max_words = (area + 3) & ~3;
-  for (int64_t t = warp0; t < num_tiles; t += nwarps) {
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * kValWarps + warp; t < num_tiles; t += nw) {
     const int64_t w0 = off[t], w1 = off[t + 1];
     bool bad = w0 < 0 || w1 < w0 || (w0 & 3) || (w1 & 3) || w1 > nwords || (w1 - w0) > max_words;
     if (t == 0 && w0 != 0) bad = true;
@@ -195,7 +203,8 @@ __global__ void __launch_bounds__(kEncThreads) tcsl_validate_kernel(const int32_
       continue;
     }
     const TileGeom g = tile_geom(t, TK, M, K, tile_m, tile_k);
-    int prev_loc = -1;          // last real loc of the previous batch
+    for (int i = lane; i < (area + 31) / 32; i += 32) seen[i] = 0u;
+    __syncwarp();
     bool seen_sentinel = false;  // a sentinel appeared in an earlier batch
     int nreal = 0;
     for (int64_t b0 = w0; b0 < w1; b0 += 32) {
@@ -208,7 +217,12 @@ __global__ void __launch_bounds__(kEncThreads) tcsl_validate_kernel(const int32_
       if (valid && sent && w != kSentinel) lane_bad = true;
       if (valid && !sent) {
         const int r = loc / tile_k, c = loc - (loc / tile_k) * tile_k;
-        if (loc >= area || r >= g.rows || c >= g.cols || (w & 0xFFFFu) == 0u) lane_bad = true;
+        if (loc >= area || r >= g.rows || c >= g.cols || (w & 0xFFFFu) == 0u) {
+          lane_bad = true;
+        } else {
+          const uint32_t bit = 1u << (loc & 31);
+          if (atomicOr(&seen[loc >> 5], bit) & bit) lane_bad = true;  // location stored twice
+        }
       }
       const uint32_t real_mask = __ballot_sync(0xFFFFFFFFu, valid && !sent);
       const uint32_t sent_mask = __ballot_sync(0xFFFFFFFFu, valid && sent);
@@ -217,17 +231,127 @@ __global__ void __launch_bounds__(kEncThreads) tcsl_validate_kernel(const int32_
         const int first_sent = __ffs(sent_mask) - 1;
         if (real_mask >> first_sent) lane_bad = true;
       }
-      int left = __shfl_up_sync(0xFFFFFFFFu, loc, 1);
-      if (lane == 0) left = prev_loc;
-      if (valid && !sent && left >= 0 && (lane == 0 || ((real_mask >> (lane - 1)) & 1u)) && loc <= left)
-        lane_bad = true;
-      if (real_mask) prev_loc = __shfl_sync(0xFFFFFFFFu, loc, 31 - __clz(real_mask));
       seen_sentinel |= sent_mask != 0u;
       nreal += __popc(real_mask);
       if (__any_sync(0xFFFFFFFFu, lane_bad)) bad = true;
     }
+    __syncwarp();
     if ((w1 - w0) - nreal >= 4) bad = true;
     if (bad && lane == 0) record_status(status, FLASHSPMM_ERR_CORRUPT_FORMAT);
+  }
+}
+
+// Word order v2 (bank-balanced), 64 x 64 tiles, one warp per tile, in place
+// on an ascending-loc encoding.  A tile's words are stored in the dense
+// shared-memory tile at byte x = 2*loc with the 128-byte swizzle
+// x ^ ((x >> 3) & 0x70), so a word's bank is bits 2-6 of that offset.  The
+// real words (before the first sentinel) are placed window by window, a
+// window being 32 consecutive positions from the tile start: at a window's
+// start the banks are ranked by unplaced words (most first, ties to the lower
+// bank), and the window takes the lowest-loc unplaced word of each bank in
+// rank order, round after round, until it is full.  In round r the banks
+// still holding more than r words are exactly the first k_r ranks, so bank b
+// of rank q places its r-th word at position k_0 + ... + k_{r-1} + q.
+constexpr int kReorderWarps = 2;
+constexpr int kReorderListWords = 4096;
+
+__device__ __forceinline__ uint32_t word_bank(uint32_t w) {
+  const uint32_t x = (w >> 15) & 0x1FFEu;  // 2 * loc for loc < 4096
+  return ((x ^ ((x >> 3) & 0x70u)) >> 2) & 31u;
+}
+
+__global__ void __launch_bounds__(kReorderWarps * 32)
+    tcsl_reorder_banks_kernel(const int32_t* __restrict__ off, uint32_t* __restrict__ words, int64_t num_tiles,
+                              int64_t nwords, int* status) {
+  __shared__ uint32_t s_list[kReorderWarps][kReorderListWords];  // the tile's words grouped by bank
+  __shared__ int s_count[kReorderWarps][32];
+  __shared__ int s_fill[kReorderWarps][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  uint32_t* list = s_list[warp];
+  int* count = s_count[warp];
+  int* fill = s_fill[warp];
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kReorderWarps;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * kReorderWarps + warp; t < num_tiles; t += nwarps) {
+    const int64_t b0 = off[t], e0 = off[t + 1];
+    const int64_t len64 = e0 - b0;
+    if (b0 < 0 || len64 < 0 || len64 > kReorderListWords || e0 > nwords || (b0 & 3) || (len64 & 3)) {
+      if (lane == 0) record_status(status, FLASHSPMM_ERR_CORRUPT_FORMAT);
+      continue;
+    }
+    const int len = static_cast<int>(len64);
+    uint32_t* tw = words + b0;
+    count[lane] = 0;
+    fill[lane] = 0;
+    __syncwarp();
+    // pass 1: the real words are those before the first sentinel; count them per bank
+    int n = len;
+    bool corrupt = false;
+    for (int i0 = 0; i0 < len; i0 += 32) {
+      const int i = i0 + lane;
+      const uint32_t w = i < len ? tw[i] : kSentinel;
+      const uint32_t sent = __ballot_sync(0xFFFFFFFFu, i < len && w == kSentinel);
+      const int stop = sent ? i0 + __ffs(sent) - 1 : len;
+      const bool real = i < len && i < stop;
+      if (real) {
+        if ((w >> 16) >= 4096u) corrupt = true;
+        else atomicAdd(&count[word_bank(w)], 1);
+      }
+      if (sent) {
+        n = stop;
+        break;
+      }
+    }
+    if (__any_sync(0xFFFFFFFFu, corrupt)) {
+      if (lane == 0) record_status(status, FLASHSPMM_ERR_CORRUPT_FORMAT);
+      continue;
+    }
+    __syncwarp();
+    const int cnt = count[lane];  // lane b: words of bank b
+    int start = cnt;              // exclusive prefix over banks: where bank b's words begin in the list
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, start, o);
+      if (lane >= o) start += y;
+    }
+    start -= cnt;
+    // pass 2: stable placement of the words into bank-major lists (ascending loc within a bank)
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const int i = i0 + lane;
+      const bool real = i < n;
+      const uint32_t w = real ? tw[i] : 0u;
+      const uint32_t bank = real ? word_bank(w) : 32u;
+      const uint32_t same = __match_any_sync(0xFFFFFFFFu, bank);
+      const int base = __shfl_sync(0xFFFFFFFFu, start, static_cast<int>(bank & 31u)) + (real ? fill[bank & 31u] : 0);
+      if (real) list[base + __popc(same & lt_mask)] = w;
+      __syncwarp();
+      // the highest lane of each bank group advances that bank's fill
+      if (real && (same >> lane) == 1u) fill[bank] += __popc(same);
+      __syncwarp();
+    }
+    // windows
+    int taken = 0;  // lane b: words of bank b placed so far
+    for (int placed = 0; placed < n;) {
+      const int room = min(32, n - placed);
+      const int rem = cnt - taken;
+      int rank = 0;  // banks with more unplaced words, or as many and a lower index
+      for (int l = 0; l < 32; ++l) {
+        const int rl = __shfl_sync(0xFFFFFFFFu, rem, l);
+        rank += (rl > rem || (rl == rem && l < lane)) ? 1 : 0;
+      }
+      int s = 0, mine = 0;
+      for (int r = 0; s < room; ++r) {
+        const int k = __popc(__ballot_sync(0xFFFFFFFFu, rem > r));
+        if (k == 0) break;  // cannot happen while the counts are consistent
+        if (rem > r && s + rank < room) {
+          tw[placed + s + rank] = list[start + taken + r];
+          ++mine;
+        }
+        s += k;
+      }
+      taken += mine;
+      placed += room;
+    }
   }
 }
 
@@ -263,12 +387,24 @@ cudaError_t launch_tcsl_fill(const void* A, int32_t M, int32_t K, int32_t tile_m
   return cudaGetLastError();
 }
 
+cudaError_t launch_tcsl_reorder_banks(const int32_t* tile_offsets, uint32_t* words, int64_t num_tiles, int64_t nwords,
+                                      cudaStream_t s) {
+  if (num_tiles == 0) return cudaSuccess;
+  const int64_t blocks = (num_tiles + kReorderWarps - 1) / kReorderWarps;
+  const int grid = static_cast<int>(max64(1, min64(blocks, 148 * 32)));
+  tcsl_reorder_banks_kernel<<<grid, kReorderWarps * 32, 0, s>>>(tile_offsets, words, num_tiles, nwords,
+                                                                device_status_ptr());
+  note_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_tcsl_validate(const flashspmm_tcsl* A, cudaStream_t s) {
   const int TK = (A->K + A->tile_k - 1) / A->tile_k;
   const int64_t nt = static_cast<int64_t>((A->M + A->tile_m - 1) / A->tile_m) * TK;
   if (nt == 0) return cudaSuccess;
-  tcsl_validate_kernel<<<enc_grid(nt), kEncThreads, 0, s>>>(A->tile_offsets, A->words, A->nwords, A->M, A->K,
-                                                           A->tile_m, A->tile_k, TK, nt, device_status_ptr());
+  const int grid = static_cast<int>(max64(1, min64((nt + kValWarps - 1) / kValWarps, 148 * 32)));
+  tcsl_validate_kernel<<<grid, kValWarps * 32, 0, s>>>(A->tile_offsets, A->words, A->nwords, A->M, A->K, A->tile_m,
+                                                       A->tile_k, TK, nt, device_status_ptr());
   note_launch();
   return cudaGetLastError();
 }
