@@ -171,10 +171,13 @@ size_t flashspmm_spmm_workspace_bytes(int32_t M, int32_t K, int32_t N, int32_t s
  *              Results are deterministic for a given (problem, split_k, device).
  *   workspace  device, >= flashspmm_spmm_workspace_bytes(...), 16-byte aligned;
  *              may be NULL when that size is 0.  Holds fp32 partial sums and
- *              per-unit arrival counters; the call clears the counters on
- *              `stream` before its kernel, so the contents need no
- *              preparation.  Calls that may run concurrently need separate
- *              workspaces.
+ *              arrival counters.  Zero it once when it is allocated: every
+ *              call that completes leaves the counters zero again (the last
+ *              arriving CTA of a unit resets its counter), so one workspace
+ *              serves any sequence of calls ordered on a stream without a
+ *              clearing step between them.  After FLASHSPMM_ERR_TIMEOUT zero
+ *              it again before reuse.  Calls that may run concurrently need
+ *              separate workspaces.
  * The kernel is launched with programmatic stream serialisation: its
  * prologue may overlap the tail of the previous kernel in the stream, and it
  * reads no input before that kernel has completed.
@@ -205,10 +208,12 @@ flashspmm_status flashspmm_spmm_lscd_host(const flashspmm_tcsl* A, const void* B
  *   - A problem whose flashspmm_spmm_workspace_bytes(M, K, N, split_k) exceeds
  *     that size returns FLASHSPMM_ERR_CAPACITY and launches nothing (with
  *     split_k = 0 on a 148-SM B200, every N <= 96 fits).
- *   - The first call on a device looks up the array's device address; make
- *     that first call before any stream capture.
- *   - All calls on a device share the one array and each call clears the
- *     arrival counters on `stream` before its kernel.
+ *   - The first call in a device's context looks up the array's device
+ *     address (cudaGetSymbolAddress, with that device current) and caches it
+ *     for that context; make that first call before any stream capture.  After
+ *     a device reset the next call looks it up again.
+ *   - All calls on a device share the one array; each call clears its
+ *     arrival counters on `stream` (cudaMemsetAsync) before its kernel.
  *     Calls that can overlap on the GPU (unordered streams) race on the array
  *     and give wrong results.
  *   - Other arguments and errors as flashspmm_spmm_lscd. */

@@ -76,8 +76,19 @@ def test_owner_and_partial_slots(M, K):
         slots = [binding.plan_slot(M, K, N, split_k, sms, pc, u) for pc, u in writers]
         assert all(0 <= s < pl["partial_slots"] for s in slots)
         assert len(set(slots)) == len(slots)
-        assert pl["workspace_bytes"] == _align256(pl["partial_slots"] * 128 * N * 4) + _align256(U * 4)
+        # a fixed 4 KB counter region (never holds partial sums, so it stays zero
+        # between calls), then the partial sums; counters that do not fit the
+        # region (explicit split-K over more than 1024 units) follow them
+        counters = pl["num_pieces"] if pl["mode"] == 0 else U
+        expect = 4096 + _align256(pl["partial_slots"] * 128 * N * 4)
+        if counters > 1024:
+            expect += _align256(counters * 4)
+        assert pl["workspace_bytes"] == expect
         if pl["mode"] == 0:
+            # a shared unit's counter is indexed by its first piece: distinct per shared unit
+            shared = sorted({u for _, u in writers})
+            firsts = [binding.plan_owner(M, K, N, split_k, sms, u * TK) for u in shared]
+            assert len(set(firsts)) == len(firsts)
             # the pieces that contribute to a unit are exactly the owners of its first..last step
             for u in range(U):
                 first = binding.plan_owner(M, K, N, split_k, sms, u * TK)

@@ -178,18 +178,19 @@ def test_workspace_too_small_is_rejected():
 
 
 @pytest.mark.parametrize("s_pct", [95, 99])
-def test_producer_far_ahead_high_sparsity(s_pct):
-    """Large, very sparse problem: the word producer runs many steps ahead of the
-    consumers, so step metadata slots are reused while earlier chunks are still
-    being consumed (a liveness case: must finish without a timeout)."""
+def test_many_short_tiles_high_sparsity(s_pct):
+    """Large, very sparse problem: every step is a partial one-batch tile, so the
+    decompress warps cycle through their staging slots and buffers far more
+    often than they expand words, and the MMA warps run many rounds per unit
+    (a liveness case: must finish without a timeout, within the bound)."""
     W, B = _case(9216, 9216, 8, s_pct, key=(212, s_pct))
     assert_parity(gpu_spmm(gpu_encode(W), B), *_oracle(W, B), f"9216^2 s={s_pct}")
 
 
 @pytest.mark.parametrize("N", [8, 64])
 def test_sparse_matrix_with_dense_tiles(N):
-    """A very sparse matrix (small load rounds) holding one fully dense 64 x 64
-    tile (4096 words: many rounds for one warp) and one dense row segment."""
+    """A very sparse matrix holding one fully dense 64 x 64 tile (4096 words:
+    sixteen full batches for one warp) and one dense row segment."""
     W, B = _case(1024, 1024, N, 95, key=(213, N))
     g = np.random.default_rng(213)
     W[128:192, 320:384] = (g.standard_normal((64, 64)) * 0.02).astype(np.float16)
@@ -221,3 +222,18 @@ def test_bank_balanced_word_order(structure, s_pct, N):
     t = fs.tcsl_encode(torch.from_numpy(W).cuda(), order=1)
     fs.check_device_status()
     assert_parity(gpu_spmm(t, B), *_oracle(W, B), f"v2 {structure} {s_pct}% N={N}")
+
+
+def test_workspace_counters_left_zero_across_plans():
+    """One workspace, zeroed once, serves calls with different plans: every
+    completed call leaves its arrival counters zero, and the partial sums of
+    one call never land where a later call keeps its counters."""
+    ws = torch.zeros(1 << 24, dtype=torch.uint8, device="cuda")
+    for M, K, N in [(4096, 4096, 32), (1024, 2048, 8), (9216, 1024, 64), (4096, 4096, 32)]:
+        W, B = _case(M, K, N, 80, key=(215, M + N))
+        need = fs.spmm_workspace_bytes(M, K, N, 0)
+        assert 4096 < need <= ws.numel()  # these shapes share units between pieces
+        C = fs.spmm_lscd(gpu_encode(W), torch.from_numpy(B).cuda(), workspace=ws)
+        fs.check_device_status()
+        assert_parity(C.cpu().numpy(), *_oracle(W, B), f"{M}x{K}x{N}")
+        assert int(ws[:4096].count_nonzero()) == 0

@@ -205,7 +205,8 @@ def _workspace(device: torch.device, nbytes: int) -> torch.Tensor | None:
     key = (device.index, )
     ws = _workspaces.get(key)
     if ws is None or ws.numel() < nbytes:
-        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        # zeroed once here; every completed call leaves its counters zero again
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
         _workspaces[key] = ws
     return ws
 

@@ -2,8 +2,11 @@
 // launchers.  This is the host wrapper the Flash-LLM review lists as
 // SpMM_API (section 5, "project structure"), reshaped as a plain C ABI that
 // takes device pointers, sizes and a stream and never allocates.
+#include <cuda.h>
+
 #include <atomic>
 #include <cstdint>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -14,19 +17,57 @@ __device__ int g_device_status = 0;
 static std::atomic<uint64_t> g_launches{0};
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
-int* device_status_ptr() {
-  static std::atomic<int*> cache[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  int* p = cache[dev].load(std::memory_order_acquire);
-  if (!p) {
-    void* a = nullptr;
-    if (cudaGetSymbolAddress(&a, g_device_status) != cudaSuccess) return nullptr;
-    p = static_cast<int*>(a);
-    cache[dev].store(p, std::memory_order_release);
-  }
-  return p;
+namespace {
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  return fn;
 }
+
+struct SymbolCache {
+  std::mutex mu;
+  CUcontext ctx[64][2] = {};
+  void* ptr[64][2] = {};
+};
+
+SymbolCache& symbol_cache() {
+  static SymbolCache c;
+  return c;
+}
+
+}  // namespace
+
+void* symbol_address_cached(int slot, const void* symbol) {
+  int dev = 0;
+  if (slot < 0 || slot > 1 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  CtxGetCurrentFn get = ctx_get_current();
+  if (!get) return nullptr;
+  CUcontext ctx = nullptr;  // null until the runtime has made the device's context current
+  if (get(&ctx) != CUDA_SUCCESS) return nullptr;
+  SymbolCache& c = symbol_cache();
+  std::lock_guard<std::mutex> lock(c.mu);
+  if (!ctx || c.ctx[dev][slot] != ctx || !c.ptr[dev][slot]) {
+    void* a = nullptr;
+    // the lookup also creates and binds the device's primary context if needed
+    if (cudaGetSymbolAddress(&a, symbol) != cudaSuccess || !a) return nullptr;
+    if (get(&ctx) != CUDA_SUCCESS || !ctx) return nullptr;
+    c.ctx[dev][slot] = ctx;
+    c.ptr[dev][slot] = a;
+  }
+  return c.ptr[dev][slot];
+}
+
+int* device_status_ptr() { return static_cast<int*>(symbol_address_cached(0, &g_device_status)); }
 
 }  // namespace flashspmm
 

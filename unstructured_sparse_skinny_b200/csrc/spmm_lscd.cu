@@ -10,11 +10,12 @@
 // buffering) is prior art; this kernel keeps the stages and maps each one to
 // sm_100a:
 //
-//   gmem2reg  -> decompress warps stream their tiles' word lists into
-//                registers with coalesced 32-bit streaming loads (consecutive
-//                words on consecutive lanes), two 256-word batches in flight
-//                per warp; each warp's tiles are consecutive in memory (see
-//                below), so its loads form one stream;
+//   gmem2reg  -> decompress warps stream their tiles' word lists into a
+//                per-warp shared-memory ring with cp.async (16 bytes per lane
+//                per copy, three 256-word batches in flight per warp, no
+//                registers held), then read each batch with conflict-free
+//                32-bit shared loads; each warp's tiles are consecutive in
+//                memory (see below), so its copies form one stream;
 //   rst_smem  -> each warp zeroes its strip's half of a 128 x 64 dense A
 //   + extract    buffer with 16-byte stores and scatters every word's value to its swizzled
 //                position (UMMA K-major 128-byte layout);
@@ -65,11 +66,14 @@ constexpr int kBarEpi = 1;                          // named barrier id of the e
 constexpr int kMinStepsPerPiece = 4;
 
 // Decompress-warp word streaming: a batch is kRB rounds of 32 words (one word
-// per lane per round) of one tile; kDepth batches are in flight per warp
-// (kDepth - 1 loading while one is expanded).
+// per lane per round) of one tile.  Batches are copied from global memory into
+// a per-warp shared-memory ring of kStage slots with cp.async (16 bytes per
+// lane per copy, no registers held while in flight); kStage - 1 batches are in
+// flight while one is expanded.
 constexpr int kRB = 8;
 constexpr int kBatchWords = kRB * 32;
-constexpr int kDepth = 3;
+constexpr int kStage = 4;
+constexpr int kStageBytes = kStage * kBatchWords * 4;  // 4 KB per decompress warp
 
 // A batch descriptor packed in 32 bits: its word count (bits 0-8), the K tile
 // of its step (bits 9-28, used to load the step's B slab) and three flags.
@@ -81,15 +85,14 @@ constexpr int32_t kMaxKTiles = 1 << 20;             // K tiles a descriptor can 
 
 template <int N_MMA>
 struct Bufs {  // dense buffers (decompress pairs) per CTA for an N bucket
-  static constexpr int value = N_MMA <= 64 ? 8 : (N_MMA == 128 ? 6 : 4);
+  static constexpr int value = N_MMA <= 32 ? 8 : (N_MMA == 64 ? 6 : (N_MMA == 128 ? 5 : 4));
 };
 
 template <int N_MMA, int ND>
 struct Cfg {
   static_assert(N_MMA == 16 || N_MMA == 32 || N_MMA == 64 || N_MMA == 128 || N_MMA == 256, "N bucket");
-  static_assert(ND % 2 == 0, "pairs are split between two MMA warps by parity");
   static constexpr int kThreads = (kWarpDec + 2 * ND) * 32;  // two decompress warps per dense buffer
-  // Two MMA warps take alternate pairs, each into its own accumulator (summed
+  // Two MMA warps take the pairs by parity, each into its own accumulator (summed
   // in a fixed order by the epilogue), so two issue chains and two
   // accumulation chains run side by side; at N = 256 one accumulator pair
   // already fills tensor memory and a single MMA warp is used.
@@ -99,7 +102,8 @@ struct Cfg {
   static constexpr int kTmemCols = 2 * kMmaWarps * N_MMA < 32 ? 32 : 2 * kMmaWarps * N_MMA;
   static constexpr uint32_t kIdesc = umma_idesc_f16_f32(kUnitRows, N_MMA);
   // shared-memory layout (offsets from a 1024-aligned base)
-  static constexpr int kOffBars = ND * kPairBytes;
+  static constexpr int kOffStage = ND * kPairBytes;              // word staging rings
+  static constexpr int kOffBars = kOffStage + 2 * ND * kStageBytes;
   static constexpr int kNumBars = 2 * ND + 4 + 1;
   static constexpr int kOffMisc = kOffBars + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
@@ -112,7 +116,7 @@ struct SpmmParams {
   int64_t nwords;
   __half* C;
   float* partials;    // [slot][N][128]
-  int32_t* counters;  // [U]
+  int32_t* counters;  // mode 0: one per piece (the first piece of a shared unit); mode 1: one per unit
   int32_t M, K, N;
   int32_t TM, TK, U;
   int64_t T;
@@ -287,8 +291,7 @@ __global__ void __launch_bounds__(Cfg<N_MMA, ND>::kThreads, 1)
         const int rounds = (sg.len + ND - 1) / ND;
         for (int r = 0; r < rounds && ok; ++r) {
 #pragma unroll
-          for (int i = 0; i < ND / Cf::kMmaWarps; ++i) {
-            const int b = m + i * Cf::kMmaWarps;
+          for (int b = m; b < ND; b += Cf::kMmaWarps) {
             if (r < chunk_begin<ND>(sg.len, b + 1) - chunk_begin<ND>(sg.len, b)) {
               if (!mbar_wait(&full[b], (fph >> b) & 1u, abort_flag, budget, p.status)) {
                 ok = false;
@@ -386,9 +389,10 @@ __global__ void __launch_bounds__(Cfg<N_MMA, ND>::kThreads, 1)
           first_pc = u * p.split;
           ncontrib = p.split;
         }
+        int32_t* const counter = p.counters + (p.mode == 0 ? first_pc : u);
         __threadfence();
         named_barrier(kBarEpi, kEpiThreads);
-        if (etid == 0) *epi_last = (atomicAdd(p.counters + u, 1) == ncontrib - 1) ? 1 : 0;
+        if (etid == 0) *epi_last = (atomicAdd(counter, 1) == ncontrib - 1) ? 1 : 0;
         named_barrier(kBarEpi, kEpiThreads);
         if (*epi_last) {
           __threadfence();
@@ -410,7 +414,7 @@ __global__ void __launch_bounds__(Cfg<N_MMA, ND>::kThreads, 1)
                 if (nc + i < p.N) p.C[static_cast<int64_t>(nc + i) * p.M + m] = __float2half_rn(acc[i]);
             }
           }
-          if (etid == 0) p.counters[u] = 0;
+          if (etid == 0) *counter = 0;  // zero again for the next call
         }
         named_barrier(kBarEpi, kEpiThreads);
       }
@@ -421,9 +425,10 @@ __global__ void __launch_bounds__(Cfg<N_MMA, ND>::kThreads, 1)
     // strip h (rows 64h .. 64h + 63) of each of the pair's steps.  The pair's
     // steps are, unit segment by unit segment, its contiguous run of K tiles,
     // so a warp's tiles follow one another in memory and its loads stream.
-    // Word lists are read in batches of up to kBatchWords words (word w of a
-    // batch on lane w % 32, round w / 32), kDepth - 1 batches ahead of the one
-    // being expanded; a batch never straddles two tiles, so every 32-word round
+    // Word lists are copied in batches of up to kBatchWords words into the
+    // warp's staging ring, kStage - 1 batches ahead of the one being expanded,
+    // and expanded word w of a batch on lane w % 32, round w / 32; a batch
+    // never straddles two tiles, so every 32-word round
     // starts on a 32-word boundary from its tile's start (the windows the
     // bank-balanced word order is built for).  The first batch of a step waits
     // until the MMAs of the buffer's previous step have retired, starts the
@@ -486,51 +491,51 @@ __global__ void __launch_bounds__(Cfg<N_MMA, ND>::kThreads, 1)
     }
     int tab_base = 0;
 
-    // ---- issue side: walks the warp's tiles and batches
+    // ---- issue side: walks the warp's tiles and batches, copying each batch
+    // into its staging slot
+    const uint32_t stage = smem_u32(bufs + Cf::kOffStage + dw * kStageBytes);
+    const uint32_t* const stage_w = reinterpret_cast<const uint32_t*>(bufs + Cf::kOffStage + dw * kStageBytes);
     int ij = 0, ipos = 0;
     int32_t ia = 0, in = 0;
     uint32_t itile = 0;
-    auto issue = [&](uint32_t& desc, uint32_t (&v)[kRB]) {
-      if (ij >= my_steps) {
-        desc = 0u;
-        return;
-      }
-      uint32_t flags = kDescValid;
-      if (ipos == 0) {
-        if (ij - tab_base == 32) {
-          tab_base += 32;
-          validate(nxt_b, nxt_e, cur_a, cur_n);
-          cur_j = nxt_j;
-          load_tab(tab_base + 32, nxt_b, nxt_e, nxt_j);
+    auto issue = [&](uint32_t& desc, int slot) {
+      if (ij < my_steps) {
+        uint32_t flags = kDescValid;
+        if (ipos == 0) {
+          if (ij - tab_base == 32) {
+            tab_base += 32;
+            validate(nxt_b, nxt_e, cur_a, cur_n);
+            cur_j = nxt_j;
+            load_tab(tab_base + 32, nxt_b, nxt_e, nxt_j);
+          }
+          const int li = ij - tab_base;
+          ia = __shfl_sync(0xFFFFFFFFu, cur_a, li);
+          in = __shfl_sync(0xFFFFFFFFu, cur_n, li);
+          itile = static_cast<uint32_t>(__shfl_sync(0xFFFFFFFFu, cur_j, li));
+          flags |= kDescFirst;
         }
-        const int li = ij - tab_base;
-        ia = __shfl_sync(0xFFFFFFFFu, cur_a, li);
-        in = __shfl_sync(0xFFFFFFFFu, cur_n, li);
-        itile = static_cast<uint32_t>(__shfl_sync(0xFFFFFFFFu, cur_j, li));
-        flags |= kDescFirst;
-      }
-      const int cnt = min(in - ipos, kBatchWords);
-      const uint32_t* src = p.words + (static_cast<int64_t>(ia) + ipos + lane);
-      if (cnt == kBatchWords) {
-#pragma unroll
-        for (int i = 0; i < kRB; ++i) v[i] = __ldcs(src + 32 * i);
+        const int cnt = min(in - ipos, kBatchWords);  // a multiple of 4 words
+        // lane l copies the 16-byte groups l and l + 32 of the batch (words 4g .. 4g + 3)
+        const uint32_t* src = p.words + (static_cast<int64_t>(ia) + ipos + 4 * lane);
+        const uint32_t dst = stage + static_cast<uint32_t>(slot * kBatchWords * 4 + lane * 16);
+        if (4 * lane < cnt) cp_async_16(dst, src);
+        if (4 * (lane + 32) < cnt) cp_async_16(dst + 512, src + 128);
+        ipos += kBatchWords;
+        if (ipos >= in) {
+          flags |= kDescLast;
+          ++ij;
+          ipos = 0;
+        }
+        desc = static_cast<uint32_t>(cnt) | ((itile & kDescTileMask) << kDescTileShift) | flags;
       } else {
-        const int lim = cnt - lane;  // lane's words in this batch: rounds i with 32 i < lim
-#pragma unroll
-        for (int i = 0; i < kRB; ++i) v[i] = 32 * i < lim ? __ldcs(src + 32 * i) : kSentinel;
+        desc = 0u;
       }
-      ipos += kBatchWords;
-      if (ipos >= in) {
-        flags |= kDescLast;
-        ++ij;
-        ipos = 0;
-      }
-      desc = static_cast<uint32_t>(cnt) | ((itile & kDescTileMask) << kDescTileShift) | flags;
+      cp_async_commit();  // one group per batch slot, empty ones included, so the counting stays uniform
     };
 
     // ---- expand side
     int pj = 0;  // index (among this pair's steps) of the step being expanded
-    auto process = [&](uint32_t desc, const uint32_t (&v)[kRB]) -> bool {
+    auto process = [&](uint32_t desc, int slot) -> bool {
       if (desc & kDescFirst) {
         // the buffer is free once the MMAs of its previous step have retired
         if (!mbar_wait(&empty[pair], static_cast<uint32_t>((pj & 1) ^ 1), abort_flag, budget, p.status)) return false;
@@ -545,13 +550,14 @@ __global__ void __launch_bounds__(Cfg<N_MMA, ND>::kThreads, 1)
         __syncwarp();
       }
       const int cnt = static_cast<int>(desc & kDescCountMask);
+      const uint32_t* sw = stage_w + slot * kBatchWords + lane;
       if (cnt == kBatchWords) {
 #pragma unroll
-        for (int i = 0; i < kRB; ++i) scatter_word(hb, v[i]);
+        for (int i = 0; i < kRB; ++i) scatter_word(hb, sw[32 * i]);
       } else {
 #pragma unroll
         for (int i = 0; i < kRB; ++i)
-          if (32 * i < cnt) scatter_word(hb, v[i]);
+          if (32 * i < cnt) scatter_word(hb, 32 * i + lane < cnt ? sw[32 * i] : kSentinel);
       }
       if (desc & kDescLast) {
         fence_proxy_async_smem();  // generic-proxy stores -> tensor-core (async proxy) reads
@@ -562,20 +568,23 @@ __global__ void __launch_bounds__(Cfg<N_MMA, ND>::kThreads, 1)
       return true;
     };
 
-    uint32_t v[kDepth][kRB];
-    uint32_t dsc[kDepth];
+    uint32_t dsc[kStage];
 #pragma unroll
-    for (int s = 0; s < kDepth - 1; ++s) issue(dsc[s], v[s]);
+    for (int s = 0; s < kStage - 1; ++s) issue(dsc[s], s);
     bool run = true;
     while (run) {
 #pragma unroll
-      for (int s = 0; s < kDepth; ++s) {
+      for (int s = 0; s < kStage; ++s) {
         if (run) {
-          issue(dsc[(s + kDepth - 1) % kDepth], v[(s + kDepth - 1) % kDepth]);
-          if (!(dsc[s] & kDescValid) || !process(dsc[s], v[s])) run = false;
+          __syncwarp();  // every lane is done reading the slot about to be refilled
+          issue(dsc[(s + kStage - 1) % kStage], (s + kStage - 1) % kStage);
+          cp_async_wait<kStage - 1>();  // this lane's copies of slot s have landed
+          __syncwarp();                 // ... and every other lane's
+          if (!(dsc[s] & kDescValid) || !process(dsc[s], s)) run = false;
         }
       }
     }
+    cp_async_wait<0>();  // no copy into shared memory outlives the CTA
     // every B slab this pair requested has landed before shared memory is
     // released (its last step's full barrier phase completed, or the wait ran
     // out of budget)
@@ -647,19 +656,20 @@ flashspmm_status launch_bucket(const flashspmm_tcsl* A, const void* B, void* C, 
   p.nwords = A->nwords;
   p.C = static_cast<__half*>(C);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  p.partials = plan.partial_bytes ? reinterpret_cast<float*>(ws) : nullptr;
-  p.counters = plan.counter_bytes ? reinterpret_cast<int32_t*>(ws + plan.partial_bytes) : nullptr;
+  p.partials = plan.partial_bytes ? reinterpret_cast<float*>(ws + plan.partial_offset) : nullptr;
+  p.counters = plan.counter_bytes ? reinterpret_cast<int32_t*>(ws + plan.counter_offset) : nullptr;
   p.M = M; p.K = K; p.N = N;
   p.TM = plan.TM; p.TK = plan.TK; p.U = plan.U; p.T = plan.T;
   p.mode = plan.mode; p.split = plan.split; p.num_pieces = plan.num_pieces;
   p.timeout_ns = 1000000000ull;  // 1 s: far above any legitimate wait
   p.status = device_status_ptr();
 
-  // The arrival counters must start at zero.  (The last arriver of a unit
-  // resets its counter, but a later call with another plan places its
-  // counters elsewhere in the workspace, possibly over partial sums left by
-  // this one, so they are cleared on the stream before every launch.)
-  if (p.counters && cudaMemsetAsync(p.counters, 0, plan.counter_bytes, s) != cudaSuccess) return FLASHSPMM_ERR_CUDA;
+  // The arrival counters must start at zero.  Counters in the fixed region at
+  // the start of the workspace are left zero by every completed call (the
+  // last arriver resets its own); the rare plans whose counters do not fit
+  // there keep them after the partial sums and clear them here.
+  if (plan.counters_cleared && cudaMemsetAsync(p.counters, 0, plan.counter_bytes, s) != cudaSuccess)
+    return FLASHSPMM_ERR_CUDA;
 
   // Programmatic stream serialisation: this kernel's prologue (barrier init,
   // tensor-memory allocation) may overlap the tail of the previous kernel in
@@ -713,10 +723,20 @@ SpmmPlan make_spmm_plan(int32_t M, int32_t K, int32_t N, int32_t split_k, int nu
     pl.num_pieces = static_cast<int32_t>(static_cast<int64_t>(pl.U) * pl.split);
     pl.partial_slots = pl.split > 1 ? pl.num_pieces : 0;
   }
-  pl.counters = pl.partial_slots ? pl.U : 0;
+  // counters: mode 0 indexes them by the first piece of a shared unit (unique
+  // per shared unit, at most one per CTA), mode 1 by unit
+  pl.counters = pl.partial_slots ? (pl.mode == 0 ? pl.num_pieces : pl.U) : 0;
   pl.partial_bytes = align256(static_cast<size_t>(pl.partial_slots) * kUnitRows * N * sizeof(float));
-  pl.counter_bytes = align256(static_cast<size_t>(pl.counters) * sizeof(int32_t));
-  pl.workspace_bytes = pl.partial_bytes + pl.counter_bytes;
+  if (pl.partial_slots == 0) {
+    pl.workspace_bytes = 0;
+    return pl;
+  }
+  pl.partial_offset = kCounterRegionBytes;
+  pl.counters_cleared = pl.counters > kCounterRegionSlots;
+  pl.counter_offset = pl.counters_cleared ? pl.partial_offset + pl.partial_bytes : 0;
+  pl.counter_bytes = pl.counters_cleared ? align256(static_cast<size_t>(pl.counters) * sizeof(int32_t))
+                                         : kCounterRegionBytes;
+  pl.workspace_bytes = pl.partial_offset + pl.partial_bytes + (pl.counters_cleared ? pl.counter_bytes : 0);
   return pl;
 }
 

@@ -8,7 +8,6 @@
 // file gives them flashspmm_spmm_lscd_noalloc, which takes its scratch from a
 // fixed-size array that the library itself places in device memory when it is
 // loaded, so the call allocates nothing.
-#include <atomic>
 #include <cstdint>
 
 #include "common.cuh"
@@ -21,20 +20,10 @@ namespace {
 static __device__ __align__(256) uint8_t g_noalloc_scratch[FLASHSPMM_NOALLOC_SCRATCH_BYTES];
 
 // In host code `g_noalloc_scratch` names a host-side stand-in, not device
-// memory; the device address is looked up once per device.
-void* noalloc_scratch_ptr() {
-  static std::atomic<void*> cache[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  void* p = cache[dev].load(std::memory_order_acquire);
-  if (!p) {
-    void* a = nullptr;
-    if (cudaGetSymbolAddress(&a, g_noalloc_scratch) != cudaSuccess || a == nullptr) return nullptr;
-    p = a;
-    cache[dev].store(p, std::memory_order_release);
-  }
-  return p;
-}
+// memory.  The device address is looked up with cudaGetSymbolAddress on the
+// first call in each context (with that device current) and cached; a device
+// reset makes a new context and so a new lookup.
+void* noalloc_scratch_ptr() { return symbol_address_cached(1, &g_noalloc_scratch); }
 
 bool aligned16_ptr(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -71,8 +60,12 @@ extern "C" flashspmm_status flashspmm_spmm_lscd_noalloc(const flashspmm_tcsl* A,
     scratch = noalloc_scratch_ptr();
     if (!scratch) return FLASHSPMM_ERR_CUDA;
   }
-  // The array keeps whatever the last call left in it.  The launcher clears
-  // the arrival counters (which must start at zero) on the stream before the
-  // kernel; the partial sums are always written before they are read.
+  // The array keeps whatever the last call left in it: clear the arrival
+  // counters (which must start at zero) on the stream before the kernel,
+  // unless the launcher clears them itself.  The partial sums are always
+  // written before they are read.
+  if (plan.counter_bytes && !plan.counters_cleared &&
+      cudaMemsetAsync(static_cast<uint8_t*>(scratch) + plan.counter_offset, 0, plan.counter_bytes, s) != cudaSuccess)
+    return FLASHSPMM_ERR_CUDA;
   return launch_spmm_lscd(A, B, C, M, K, N, plan, scratch, s);
 }
