@@ -10,37 +10,37 @@
 // buffering) is prior art; this kernel keeps the stages and maps each one to
 // sm_100a:
 //
-//   gmem2reg  -> decompress warps stream their tiles' word lists into a
-//                per-warp shared-memory ring with cp.async (16 bytes per lane
-//                per copy, three 256-word batches in flight per warp, no
-//                registers held), then read each batch with conflict-free
-//                32-bit shared loads; each warp's tiles are consecutive in
-//                memory (see below), so its copies form one stream;
-//   rst_smem  -> each warp zeroes its strip's half of a 128 x 64 dense A
-//   + extract    buffer with 16-byte stores and scatters every word's value to its swizzled
-//                position (UMMA K-major 128-byte layout);
-//   ld_dense  -> each step's B slab (64 K x N_MMA) is loaded by TMA into the
-//                step's buffer in the same swizzled layout, completing on the
-//                barrier that hands the step to the MMA warps;
+//   gmem2reg  -> 8 decompress warps stream their tiles' word lists from HBM
+//                straight into registers (coalesced 32-bit loads, L1
+//                bypassed, L2 evict-first), one round (1024 words, or 512
+//                for very sparse matrices) always in flight per warp while
+//                the previous round is expanded;
+//   rst_smem  -> each warp zeroes its half (64 rows) of a 128 x 64 dense A
+//   + extract    buffer with 16-byte stores and scatters every word's value
+//                to its swizzled position (UMMA K-major 128-byte layout);
+//   ld_dense  -> warp 1 loads B slabs (64 K x N_MMA) with TMA tensor copies in
+//                the same swizzled layout, several K tiles per request;
 //   smem2tc   -> gone: tcgen05.mma reads both operands from shared memory;
-//   TC_compute-> two MMA warps issue 4 x tcgen05.mma (M = 128, K = 16) per step
-//                into double-buffered fp32 accumulators in tensor memory;
+//   TC_compute-> warp 0 issues 4 x tcgen05.mma (M = 128, K = 16) per step into
+//                a double-buffered fp32 accumulator in tensor memory;
 //   epilogue  -> 4 warps read the accumulator with tcgen05.ld and write fp16 C
 //                (or fp32 partial sums, see below).
 //
 // A "unit" is 128 rows of A (two 64-row format strips stacked on the MMA M
-// side); a "step" is one 64-wide K tile of one unit.  Each pair of decompress
-// warps owns one buffer (16 KB dense A tile + B slab) and expands its share of
-// the CTA's steps into it, one warp per strip: two mbarrier arrivals and the
-// B slab's bytes hand the step to the MMA warps, one tcgen05.commit hands the
-// buffer back.  No pair waits on another pair.
+// side); a "step" is one 64-wide K tile of one unit, expanded by a pair of
+// decompress warps (one per strip) into a dense buffer.  The CTA's steps are
+// taken in groups of 4; pair p expands step p of every group, and the groups
+// alternate between two sets of 4 dense buffers.  A group costs one mbarrier
+// hand-off (8 arrivals) to the MMA warp and one commit back, which the MMA
+// warp answers with 16 MMAs: per-step synchronisation, not data, is what
+// limits a skinny SpMM, so it is paid once per group.
 //
 // The T = units x K-tiles steps are cut into contiguous pieces, one CTA each.
 // When a unit is shared by several pieces, every piece writes its fp32
 // partial sum to the workspace and the last piece to finish (atomic arrival
 // counter) adds them in piece order and writes C: the split-K reduction of the
 // page's Reduction kernel (section 5, "project structure"), fused and
-// deterministic.
+// deterministic.  The last piece also resets the unit's arrival counter.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
@@ -55,56 +55,38 @@ namespace {
 
 constexpr int kTile = 64;                           // format tile edge (rows and K)
 constexpr int kUnitRows = 128;                      // MMA M
-constexpr int kDenseBytes = kUnitRows * kTile * 2;  // 16 KB dense A buffer (one step)
+constexpr int kDenseBytes = kUnitRows * kTile * 2;  // 16 KB dense A buffer
 constexpr int kHalfBytes = kDenseBytes / 2;         // one strip's 64 rows
 constexpr int kMaxTileWords = kTile * kTile;        // 4096 words (already a multiple of 4)
-// Warp roles: MMA issuers (warps 0 and 1), epilogue (2-5, one per
-// tensor-memory lane quarter), decompress warps (6 and up, in pairs).
-constexpr int kWarpMma = 0, kWarpMma1 = 1, kWarpEpi = 2, kWarpDec = 6;
+constexpr int kWarpMma = 0, kWarpB = 1, kWarpEpi = 2, kWarpDec = 6;
+constexpr int kDecWarps = 8;                        // 4 pairs, one warp per strip
+constexpr int kPairs = kDecWarps / 2;
+constexpr int kThreads = (kWarpDec + kDecWarps) * 32;
 constexpr int kEpiThreads = 128;
+constexpr int kNumDense = 2 * kPairs;               // two sets of one buffer per pair
 constexpr int kBarEpi = 1;                          // named barrier id of the epilogue warps
+// Words per lane per load round (a round is 32x that per warp): 32 for most
+// matrices, 16 when a tile averages at most kSmallRoundMaxWords words, where
+// 32-word rounds would be mostly sentinel slots that still cost instructions.
+constexpr int kRoundRegsLarge = 32, kRoundRegsSmall = 16;
+constexpr int kSmallRoundMaxWords = 448;
 constexpr int kMinStepsPerPiece = 4;
 
-// Decompress-warp word streaming: a batch is kRB rounds of 32 words (one word
-// per lane per round) of one tile.  Batches are copied from global memory into
-// a per-warp shared-memory ring of kStage slots with cp.async (16 bytes per
-// lane per copy, no registers held while in flight); kStage - 1 batches are in
-// flight while one is expanded.
-constexpr int kRB = 8;
-constexpr int kBatchWords = kRB * 32;
-constexpr int kStage = 4;
-constexpr int kStageBytes = kStage * kBatchWords * 4;  // 4 KB per decompress warp
-
-// A batch descriptor packed in 32 bits: its word count (bits 0-8), the K tile
-// of its step (bits 9-28, used to load the step's B slab) and three flags.
-constexpr uint32_t kDescCountMask = (1u << 9) - 1u;
-constexpr int kDescTileShift = 9;
-constexpr uint32_t kDescTileMask = (1u << 20) - 1u;
-constexpr uint32_t kDescValid = 1u << 29, kDescFirst = 1u << 30, kDescLast = 1u << 31;
-constexpr int32_t kMaxKTiles = 1 << 20;             // K tiles a descriptor can name
 
 template <int N_MMA>
-struct Bufs {  // dense buffers (decompress pairs) per CTA for an N bucket
-  static constexpr int value = N_MMA <= 32 ? 8 : (N_MMA == 64 ? 6 : (N_MMA == 128 ? 5 : 4));
-};
-
-template <int N_MMA, int ND>
 struct Cfg {
   static_assert(N_MMA == 16 || N_MMA == 32 || N_MMA == 64 || N_MMA == 128 || N_MMA == 256, "N bucket");
-  static constexpr int kThreads = (kWarpDec + 2 * ND) * 32;  // two decompress warps per dense buffer
-  // Two MMA warps take the pairs by parity, each into its own accumulator (summed
-  // in a fixed order by the epilogue), so two issue chains and two
-  // accumulation chains run side by side; at N = 256 one accumulator pair
-  // already fills tensor memory and a single MMA warp is used.
-  static constexpr int kMmaWarps = N_MMA <= 128 ? 2 : 1;
-  static constexpr int kBSlabBytes = N_MMA * kTile * 2;   // one 64-wide K tile of B (N_MMA rows)
-  static constexpr int kPairBytes = kDenseBytes + kBSlabBytes;  // a pair's dense A tile + its B slab
-  static constexpr int kTmemCols = 2 * kMmaWarps * N_MMA < 32 ? 32 : 2 * kMmaWarps * N_MMA;
+  static constexpr int kBSlabBytes = N_MMA * kTile * 2;  // one 64-wide K tile of B
+  static constexpr int kSlabsPerReq = kBSlabBytes >= 16384 ? 1 : 16384 / kBSlabBytes;  // K tiles per TMA request
+  static constexpr int kReqBytes = kSlabsPerReq * kBSlabBytes;
+  static constexpr int kNumReq = N_MMA <= 128 ? 3 : 2;   // B requests in flight
+  static constexpr int kTmemCols = 2 * N_MMA < 32 ? 32 : 2 * N_MMA;
   static constexpr uint32_t kIdesc = umma_idesc_f16_f32(kUnitRows, N_MMA);
   // shared-memory layout (offsets from a 1024-aligned base)
-  static constexpr int kOffStage = ND * kPairBytes;              // word staging rings
-  static constexpr int kOffBars = kOffStage + 2 * ND * kStageBytes;
-  static constexpr int kNumBars = 2 * ND + 4 + 1;
+  static constexpr int kOffDense = 0;
+  static constexpr int kOffB = kOffDense + kNumDense * kDenseBytes;
+  static constexpr int kOffBars = kOffB + kNumReq * kReqBytes;
+  static constexpr int kNumBars = 2 * 2 + 2 * kNumReq + 4 + 1;
   static constexpr int kOffMisc = kOffBars + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -121,6 +103,8 @@ struct SpmmParams {
   int32_t TM, TK, U;
   int64_t T;
   int32_t mode, split, num_pieces;
+  int32_t b_kb;    // K tiles of B per TMA request (1 with the 2-D map)
+  int32_t b_3d;    // B tensor map is 3-D (64 x N x K/64)
   uint64_t timeout_ns;
   int* status;
 };
@@ -146,30 +130,6 @@ __host__ __device__ __forceinline__ int64_t partial_slot(const SpmmParams& p, in
   return 2 * pc + ((piece_range(p, pc).b / p.TK) != u ? 1 : 0);
 }
 
-// A piece is walked unit by unit: its segment in unit u covers K tiles
-// [j0, j1), and pair b of the CTA expands the contiguous run
-// [j0 + b*L/ND, j0 + (b+1)*L/ND) of it (L = j1 - j0), so each decompress warp
-// streams a contiguous range of its strip's words.  The MMA warps take the
-// pairs' steps round robin (round r: the r-th step of pairs 0, 1, ...), a
-// fixed order, so results are deterministic.
-struct Segment {
-  int64_t u;
-  int j0, len;
-};
-
-__device__ __forceinline__ Segment segment_at(const SpmmParams& p, const Range& rg, int64_t q) {
-  Segment sg;
-  sg.u = q / p.TK;
-  sg.j0 = static_cast<int>(q - sg.u * p.TK);
-  sg.len = static_cast<int>(min64(rg.e - sg.u * p.TK, p.TK)) - sg.j0;
-  return sg;
-}
-
-template <int ND>
-__host__ __device__ __forceinline__ int chunk_begin(int len, int b) {
-  return b * len / ND;
-}
-
 __device__ __forceinline__ bool named_barrier_or(uint32_t id, uint32_t nthreads, bool pred) {
   uint32_t r;
   asm volatile(
@@ -189,8 +149,20 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
-// Words are read with streaming loads (ld.global.cs: evict-first, every word
-// is used exactly once).
+// Word `slot` of this lane in a load round, or the sentinel when the slot is
+// past the lane's `nvalid` words (the address is then not dereferenced).
+// Read-only path, no L1 allocation, evict-first in L2: every word is used
+// exactly once.
+__device__ __forceinline__ uint32_t ldg_word(const uint32_t* ptr, int slot, int nvalid, uint64_t policy) {
+  uint32_t v = kSentinel;
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.lt.s32 q, %2, %3;\n\t"
+      "@q ld.global.nc.L1::no_allocate.L2::cache_hint.b32 %0, [%1], %4;\n\t}"
+      : "+r"(v)
+      : "l"(ptr), "r"(slot), "r"(nvalid), "l"(policy));
+  return v;
+}
 
 // Writes one word's value into a strip's 64 x 64 half of the dense buffer at
 // its swizzled place.  loc = r*64 + c; the unswizzled byte offset is
@@ -208,24 +180,29 @@ __device__ __forceinline__ void scatter_word(uint32_t half_u32, uint32_t w) {
       "r"(w));
 }
 
-// A word range [b, e) from the tile offsets is usable iff it lies inside the
-// word array, starts on a 16-byte boundary and holds at most one tile.
-__device__ __forceinline__ bool range_ok(int32_t b, int32_t e, int64_t nwords) {
-  const int32_t n = e - b;
-  return b >= 0 && n >= 0 && !(b & 3) && !(n & 3) && n <= kMaxTileWords && e <= nwords;
-}
+// A load round of a decompress warp: words [base, end) of one strip tile,
+// at most 32 * RR of them.
+struct Round {
+  int k;      // index of the step among the warp's steps
+  bool first, last, valid;
+};
 
-template <int N_MMA, int ND>
-__global__ void __launch_bounds__(Cfg<N_MMA, ND>::kThreads, 1)
+template <int N_MMA, int RR>
+__global__ void __launch_bounds__(kThreads, 1)
     spmm_lscd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_b, const SpmmParams p) {
-  using Cf = Cfg<N_MMA, ND>;
+  using Cf = Cfg<N_MMA>;
+  constexpr int kRoundRegs = RR;
+  constexpr int kRoundWords = RR * 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* bufs = smem;  // ND x (dense A tile, B slab)
+  uint8_t* dense = smem + Cf::kOffDense;
+  uint8_t* bslab = smem + Cf::kOffB;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cf::kOffBars);
-  uint64_t* full = bars;             // [ND]: step expanded (one arrival per strip + the B slab's bytes)
-  uint64_t* empty = full + ND;       // [ND]: step consumed (one commit)
-  uint64_t* acc_full = empty + ND;   // [2]: accumulators of a unit complete (one commit per MMA warp)
+  uint64_t* a_full = bars;          // [2]: buffer set filled (8 arrivals)
+  uint64_t* a_empty = a_full + 2;   // [2]: buffer set consumed (one commit)
+  uint64_t* b_full = a_empty + 2;
+  uint64_t* b_empty = b_full + Cf::kNumReq;
+  uint64_t* acc_full = b_empty + Cf::kNumReq;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* mma_done = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::kOffMisc);
@@ -237,17 +214,21 @@ __global__ void __launch_bounds__(Cfg<N_MMA, ND>::kThreads, 1)
   const uint64_t budget = p.timeout_ns;
 
   griddep_launch_dependents();
-  if (warp == kWarpMma1) {
-    if (lane < ND) {
-      mbar_init(&full[lane], 2);  // both strips of the step (the B slab adds its bytes)
-      mbar_init(&empty[lane], 1);
+  if (warp == kWarpB) {
+    if (lane < 2) {
+      mbar_init(&a_full[lane], kDecWarps);  // every decompress warp, once per group
+      mbar_init(&a_empty[lane], 1);
+    }
+    if (lane < Cf::kNumReq) {
+      mbar_init(&b_full[lane], 1);
+      mbar_init(&b_empty[lane], 1);
     }
     if (lane < 2) {
-      mbar_init(&acc_full[lane], Cf::kMmaWarps);  // one commit per MMA warp
+      mbar_init(&acc_full[lane], 1);
       mbar_init(&acc_empty[lane], 1);
     }
     if (lane == 0) {
-      mbar_init(mma_done, Cf::kMmaWarps);
+      mbar_init(mma_done, 1);
       *abort_flag = 0;
       *epi_last = 0;
       prefetch_tensor_map(&tmap_b);
@@ -266,66 +247,112 @@ __global__ void __launch_bounds__(Cfg<N_MMA, ND>::kThreads, 1)
   // the previous kernel in the stream may have written) are read.
   griddep_wait();
 
-  if (warp == kWarpMma || warp == kWarpMma1) {
-    // ------------------------------------------------ tcgen05 MMA issuers
-    // MMA warp m issues the steps of pairs b with b % kMmaWarps == m, in the
-    // round-robin order, into its own accumulator of the unit.  Every lane
-    // tests the barriers itself (no broadcast needed) and one elected lane
-    // issues the MMAs and commits (issue from a converged warp is markedly
-    // cheaper than from a lone divergent thread).
-    const int m = warp == kWarpMma ? 0 : 1;
-    if (m < Cf::kMmaWarps) {
-      const bool leader = elect_one();
-      int ac = 0;          // accumulator pair of the current unit
-      uint32_t acph = 1;   // parity to wait on acc_empty[ac]
-      uint32_t fph = 0;    // bit b: parity to wait on full[b]
-      const uint64_t desc0 = smem_desc_k_sw128(smem_u32(bufs));
-      const uint32_t tmem_m = tmem_base + static_cast<uint32_t>(m * N_MMA);
-      bool ok = true;
-      for (int64_t q = rg.b; q < rg.e && ok;) {
-        const Segment sg = segment_at(p, rg, q);
-        if (!mbar_wait(&acc_empty[ac], acph, abort_flag, budget, p.status)) break;
-        tc_fence_after_sync();  // accumulator handed back by the epilogue's tcgen05.ld
-        const uint32_t tmem_d = tmem_m + static_cast<uint32_t>(ac * Cf::kMmaWarps * N_MMA);
-        uint32_t acc_flag = 0u;  // 0 until this warp's first MMA of the unit
-        const int rounds = (sg.len + ND - 1) / ND;
-        for (int r = 0; r < rounds && ok; ++r) {
-#pragma unroll
-          for (int b = m; b < ND; b += Cf::kMmaWarps) {
-            if (r < chunk_begin<ND>(sg.len, b + 1) - chunk_begin<ND>(sg.len, b)) {
-              if (!mbar_wait(&full[b], (fph >> b) & 1u, abort_flag, budget, p.status)) {
-                ok = false;
-                break;
-              }
-              fph ^= 1u << b;
-              if (leader) {
-                // descriptor start addresses advance in 16-byte units; K = 16
-                // per MMA advances 32 bytes (2 units) inside the swizzle atom
-                const uint64_t adesc = desc0 + static_cast<uint64_t>((b * Cf::kPairBytes) >> 4);
-                const uint64_t bdesc = adesc + static_cast<uint64_t>(kDenseBytes >> 4);
-                umma_f16_ss(tmem_d, adesc, bdesc, Cf::kIdesc, acc_flag);
-#pragma unroll
-                for (int kk = 1; kk < kTile / 16; ++kk)
-                  umma_f16_ss(tmem_d, adesc + 2 * kk, bdesc + 2 * kk, Cf::kIdesc, 1u);
-                umma_commit(&empty[b]);
-              }
-              acc_flag = 1u;
-            }
-          }
+  if (warp == kWarpB) {
+    // ------------------------------------------------ dense B producer (TMA)
+    // A request loads b_kb consecutive 64-wide K tiles of B (one group); the
+    // requests of the piece are the (unit, group) pairs it touches, and lane r
+    // issues every kNumReq-th request into request slot r.
+    if (lane < Cf::kNumReq) {
+      const int kb = p.b_kb;
+      const int ngroups = (p.TK + kb - 1) / kb;
+      int64_t u = rg.b / p.TK;
+      int g = static_cast<int>(rg.b - u * p.TK) / kb;
+      int64_t k = 0, uses = 0;
+      while (u * p.TK + static_cast<int64_t>(g) * kb < rg.e) {
+        if (static_cast<int>(k % Cf::kNumReq) == lane) {
+          if (!mbar_wait(&b_empty[lane], static_cast<uint32_t>((uses & 1) ^ 1), abort_flag, budget, p.status)) break;
+          mbar_arrive_expect_tx(&b_full[lane], static_cast<uint32_t>(kb * Cf::kBSlabBytes));
+          uint8_t* dst = bslab + lane * Cf::kReqBytes;
+          if (p.b_3d) tma_load_3d(dst, &tmap_b, 0, 0, g * kb, &b_full[lane]);
+          else tma_load_2d(dst, &tmap_b, g * kTile, 0, &b_full[lane]);
+          ++uses;
         }
-        if (!ok) break;
-        if (leader) umma_commit(&acc_full[ac]);
-        __syncwarp();
-        if (ac == 1) acph ^= 1u;
-        ac ^= 1;
-        q = (sg.u + 1) * p.TK;
+        ++k;
+        if (++g == ngroups) { g = 0; ++u; }
       }
-      // all MMAs of both warps retired before tensor memory is released
-      if (leader) umma_commit(mma_done);
-      __syncwarp();
-      if (lane == 0) mbar_wait_drain(mma_done, 0, budget, p.status);
+      // every issued copy lands before the CTA's shared memory is released
+      if (uses > 0) mbar_wait_drain(&b_full[lane], static_cast<uint32_t>((uses - 1) & 1), budget, p.status);
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------ tcgen05 MMA issuer
+    // The whole warp runs one uniform loop, one group of up to 4 steps per
+    // iteration; every lane tests the barriers itself (so no broadcast is
+    // needed) and one elected lane issues the MMAs and commits (issue from a
+    // converged warp is markedly cheaper than from a lone divergent thread).
+    // Before a step that starts a B request or an accumulator the warp waits
+    // for that too, never earlier: a request slot or accumulator may only be
+    // freed by this group's own earlier MMAs.  Step bookkeeping is kept in
+    // 32-bit counters: this loop is latency-bound, one iteration per group.
+    const int kb = p.b_kb;
+    int nleft = static_cast<int>(rg.e - rg.b);        // steps left in the piece
+    int to_unit = p.TK - static_cast<int>(rg.b % p.TK);  // steps left in the current unit
+    int jk = (p.TK - to_unit) % kb;                   // slab of the current step in its B request
+    bool pfirst = true;
+    int r = Cf::kNumReq - 1;  // B request slot of the current step
+    uint32_t rph = 1;         // its phase parity (flips when the slot index wraps to 0)
+    int ac = 0;               // accumulator of the current unit
+    uint32_t acph = 1;        // parity to wait on acc_empty[ac]
+    const uint32_t a_base = smem_u32(dense);
+    const uint32_t b_base = smem_u32(bslab);
+    bool issued = false, dead = false;
+    for (int64_t k = 0; nleft > 0 && !dead; ++k) {
+      const int set = static_cast<int>(k & 1);
+      if (!mbar_wait(&a_full[set], static_cast<uint32_t>((k >> 1) & 1), abort_flag, budget, p.status)) break;
+      const bool leader = elect_one();
+      const int gsteps = nleft < kPairs ? nleft : kPairs;
+#pragma unroll
+      for (int i = 0; i < kPairs; ++i) {
+        if (i >= gsteps) break;
+        const bool first = pfirst || to_unit == p.TK;
+        const bool last = nleft == 1 || to_unit == 1;
+        const bool new_req = pfirst || jk == 0;
+        if (new_req) {
+          if (++r == Cf::kNumReq) { r = 0; rph ^= 1u; }
+          if (!mbar_wait(&b_full[r], rph, abort_flag, budget, p.status)) { dead = true; break; }
+        }
+        if (first) {
+          if (!mbar_wait(&acc_empty[ac], acph, abort_flag, budget, p.status)) { dead = true; break; }
+          tc_fence_after_sync();  // accumulator handed back by the epilogue's tcgen05.ld
+        }
+        const uint64_t adesc = smem_desc_k_sw128(a_base + static_cast<uint32_t>((i + kPairs * set) * kDenseBytes));
+        const uint64_t bdesc =
+            smem_desc_k_sw128(b_base + static_cast<uint32_t>(r * Cf::kReqBytes + jk * Cf::kBSlabBytes));
+        const uint32_t tmem_d = tmem_base + static_cast<uint32_t>(ac * N_MMA);
+        uint64_t ad[kTile / 16], bd[kTile / 16];  // K = 16 per MMA: advance 32 bytes inside the swizzle atom
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) { ad[kk] = adesc + 2 * kk; bd[kk] = bdesc + 2 * kk; }
+        const uint32_t acc0 = first ? 0u : 1u;
+        if (leader) {
+          umma_f16_ss(tmem_d, ad[0], bd[0], Cf::kIdesc, acc0);
+#pragma unroll
+          for (int kk = 1; kk < kTile / 16; ++kk) umma_f16_ss(tmem_d, ad[kk], bd[kk], Cf::kIdesc, 1u);
+          if (jk == kb - 1 || last) umma_commit(&b_empty[r]);  // request fully used
+          if (last) umma_commit(&acc_full[ac]);
+        }
+        issued = true;
+        pfirst = false;
+        --nleft;
+        if (last) {
+          if (ac == 1) acph ^= 1u;
+          ac ^= 1;
+        }
+        if (--to_unit == 0) {
+          to_unit = p.TK;
+          jk = 0;
+        } else if (++jk == kb) {
+          jk = 0;
+        }
+      }
+      if (dead) break;
+      if (leader) umma_commit(&a_empty[set]);
       __syncwarp();
     }
+    if (issued) {  // all MMAs retired before tensor memory is released
+      if (elect_one()) umma_commit(mma_done);
+      __syncwarp();
+      if (lane == 0) mbar_wait_drain(mma_done, 0, budget, p.status);
+    }
+    __syncwarp();
   } else if (warp >= kWarpEpi && warp < kWarpEpi + 4) {
     // ------------------------------------------------ epilogue
     const int etid = threadIdx.x - kWarpEpi * 32;
@@ -342,32 +369,20 @@ __global__ void __launch_bounds__(Cfg<N_MMA, ND>::kThreads, 1)
       const int64_t seg_b = max64(rg.b, u * p.TK), seg_e = min64(rg.e, (u + 1) * p.TK);
       const bool complete = seg_b == u * p.TK && seg_e == (u + 1) * p.TK;
       const int64_t m = u * kUnitRows + row;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             static_cast<uint32_t>(ab * Cf::kMmaWarps * N_MMA);
-      // MMA warp w wrote its accumulator iff one of its pairs (b % kMmaWarps
-      // == w) had a step in the segment
-      const int len = static_cast<int>(seg_e - seg_b);
-      bool has0 = false, has1 = false;
-#pragma unroll
-      for (int b = 0; b < ND; ++b) {
-        const bool any = chunk_begin<ND>(len, b + 1) > chunk_begin<ND>(len, b);
-        if (Cf::kMmaWarps == 1 || (b & 1) == 0) has0 |= any;
-        else has1 |= any;
-      }
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(ab * N_MMA);
       float* part = nullptr;
       if (!complete) part = p.partials + partial_slot(p, blockIdx.x, u) * static_cast<int64_t>(p.N) * kUnitRows;
 #pragma unroll 1
-      for (int c = 0; c < N_MMA && c < p.N; c += 8) {
-        uint32_t v[8], w[8];
-        if (has0) tmem_load_8(taddr + c, v);
-        if (has1) tmem_load_8(taddr + N_MMA + c, w);
+      for (int c = 0; c < N_MMA && c < p.N; c += 16) {
+        uint32_t v[16];
+        tmem_load_16(taddr + c, v);
         tmem_load_wait();
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 16; ++i) {
           const int nn = c + i;
           if (nn < p.N) {
-            const float x = has0 && has1 ? __uint_as_float(v[i]) + __uint_as_float(w[i])
-                                         : __uint_as_float(has0 ? v[i] : w[i]);
+            const float x = __uint_as_float(v[i]);
             if (complete) {
               if (m < p.M) p.C[static_cast<int64_t>(nn) * p.M + m] = __float2half_rn(x);
             } else {
@@ -397,20 +412,20 @@ __global__ void __launch_bounds__(Cfg<N_MMA, ND>::kThreads, 1)
         if (*epi_last) {
           __threadfence();
 #pragma unroll 1
-          for (int nc = 0; nc < p.N; nc += 8) {
-            float acc[8];
+          for (int nc = 0; nc < p.N; nc += 16) {
+            float acc[16];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
 #pragma unroll 1
             for (int64_t k = 0; k < ncontrib; ++k) {
               const float* src = p.partials + (partial_slot(p, first_pc + k, u) * p.N + nc) * kUnitRows + row;
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
+              for (int i = 0; i < 16; ++i)
                 if (nc + i < p.N) acc[i] += __ldcg(src + i * kUnitRows);
             }
             if (m < p.M) {
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
+              for (int i = 0; i < 16; ++i)
                 if (nc + i < p.N) p.C[static_cast<int64_t>(nc + i) * p.M + m] = __float2half_rn(acc[i]);
             }
           }
@@ -421,174 +436,124 @@ __global__ void __launch_bounds__(Cfg<N_MMA, ND>::kThreads, 1)
     }
   } else {
     // ------------------------------------------------ decompress (gmem2reg + rst_smem + extract)
-    // Pair b owns buffer b (dense A tile + B slab); warp h of the pair expands
-    // strip h (rows 64h .. 64h + 63) of each of the pair's steps.  The pair's
-    // steps are, unit segment by unit segment, its contiguous run of K tiles,
-    // so a warp's tiles follow one another in memory and its loads stream.
-    // Word lists are copied in batches of up to kBatchWords words into the
-    // warp's staging ring, kStage - 1 batches ahead of the one being expanded,
-    // and expanded word w of a batch on lane w % 32, round w / 32; a batch
-    // never straddles two tiles, so every 32-word round
-    // starts on a 32-word boundary from its tile's start (the windows the
-    // bank-balanced word order is built for).  The first batch of a step waits
-    // until the MMAs of the buffer's previous step have retired, starts the
-    // TMA load of the step's B slab (warp 0 of the pair) and zeroes the warp's
-    // half; the last one publishes the half to the MMA warps.
+    // Warp (pair, h) expands strip h of step `pair` of every group, i.e. the
+    // steps pair, pair + 4, ... of the piece, into buffer pair of the group's
+    // buffer set.  Its word lists are streamed in rounds of up to 32 * RR words
+    // (RR per lane, consecutive words on consecutive lanes); the loads of the next
+    // round are issued before the current round is expanded, so one round is
+    // always in flight.  The first round of a step waits until the MMAs of
+    // the buffer's previous step have retired and zeroes the warp's half of
+    // the buffer; the last round publishes the half to the MMA warp.
     const int dw = warp - kWarpDec;
     const int pair = dw >> 1, h = dw & 1;
-    uint8_t* const pbuf = bufs + pair * Cf::kPairBytes;
-    const uint32_t hb = smem_u32(pbuf + h * kHalfBytes);
-    // k-th step of this pair: its unit and K tile (false past the last step)
-    auto step_of = [&](int k, int64_t& u, int& j) -> bool {
-      for (int64_t q = rg.b; q < rg.e;) {
-        const Segment sg = segment_at(p, rg, q);
-        const int c0 = chunk_begin<ND>(sg.len, pair), c1 = chunk_begin<ND>(sg.len, pair + 1);
-        if (k < c1 - c0) {
-          u = sg.u;
-          j = sg.j0 + c0 + k;
-          return true;
-        }
-        k -= c1 - c0;
-        q = (sg.u + 1) * p.TK;
-      }
-      return false;
-    };
-    int my_steps = 0;
-    for (int64_t q = rg.b; q < rg.e;) {
-      const Segment sg = segment_at(p, rg, q);
-      my_steps += chunk_begin<ND>(sg.len, pair + 1) - chunk_begin<ND>(sg.len, pair);
-      q = (sg.u + 1) * p.TK;
-    }
-    // Raw tile offsets (begin, end) and K tile of 32 consecutive steps of this
-    // warp, one step per lane.
-    auto load_tab = [&](int k0, int32_t& ob, int32_t& oe, int32_t& oj) {
-      ob = oe = oj = 0;
-      int64_t u;
-      int j;
-      if (step_of(k0 + lane, u, j)) {
-        oj = j;
-        if (2 * u + h < p.TM) {
-          const int64_t t = (2 * u + h) * p.TK + j;
-          ob = __ldg(p.tile_offsets + t);
-          oe = __ldg(p.tile_offsets + t + 1);
+    const int64_t piece_steps = rg.e - rg.b;
+    const int64_t my_steps = piece_steps > pair ? (piece_steps - pair + kPairs - 1) / kPairs : 0;
+    const uint64_t policy = l2_policy_evict_first();
+    // Tile offsets of 32 consecutive steps of this warp, one step per lane:
+    // the current table (validated) and the next one (loads in flight).
+    auto load_tab = [&](int64_t k0, int32_t& ta, int32_t& tb) {
+      ta = 0;
+      tb = 0;
+      const int64_t k = k0 + lane;
+      if (k < my_steps) {
+        const int64_t q = rg.b + pair + k * kPairs;
+        const int64_t u = q / p.TK, j = q - (q / p.TK) * p.TK;
+        const int64_t strip = 2 * u + h;
+        if (strip < p.TM) {
+          const int64_t t = strip * p.TK + j;
+          ta = __ldg(p.tile_offsets + t);
+          tb = __ldg(p.tile_offsets + t + 1);
         }
       }
     };
-    // Turns a raw (begin, end) into (start, length); a range that breaks the
-    // format is reported and replaced by an empty tile.
-    auto validate = [&](int32_t ob, int32_t oe, int32_t& ca, int32_t& cn) {
-      const bool ok = range_ok(ob, oe, p.nwords);
-      ca = ok ? ob : 0;
-      cn = ok ? oe - ob : 0;
-      if (!ok) record_status(p.status, FLASHSPMM_ERR_CORRUPT_FORMAT);
-    };
-    int32_t cur_a, cur_n, cur_j, nxt_b, nxt_e, nxt_j;
-    {
-      int32_t ob, oe;
-      load_tab(0, ob, oe, cur_j);
-      load_tab(32, nxt_b, nxt_e, nxt_j);
-      validate(ob, oe, cur_a, cur_n);
-    }
-    int tab_base = 0;
-
-    // ---- issue side: walks the warp's tiles and batches, copying each batch
-    // into its staging slot
-    const uint32_t stage = smem_u32(bufs + Cf::kOffStage + dw * kStageBytes);
-    const uint32_t* const stage_w = reinterpret_cast<const uint32_t*>(bufs + Cf::kOffStage + dw * kStageBytes);
-    int ij = 0, ipos = 0;
-    int32_t ia = 0, in = 0;
-    uint32_t itile = 0;
-    auto issue = [&](uint32_t& desc, int slot) {
-      if (ij < my_steps) {
-        uint32_t flags = kDescValid;
-        if (ipos == 0) {
-          if (ij - tab_base == 32) {
-            tab_base += 32;
-            validate(nxt_b, nxt_e, cur_a, cur_n);
-            cur_j = nxt_j;
-            load_tab(tab_base + 32, nxt_b, nxt_e, nxt_j);
-          }
-          const int li = ij - tab_base;
-          ia = __shfl_sync(0xFFFFFFFFu, cur_a, li);
-          in = __shfl_sync(0xFFFFFFFFu, cur_n, li);
-          itile = static_cast<uint32_t>(__shfl_sync(0xFFFFFFFFu, cur_j, li));
-          flags |= kDescFirst;
-        }
-        const int cnt = min(in - ipos, kBatchWords);  // a multiple of 4 words
-        // lane l copies the 16-byte groups l and l + 32 of the batch (words 4g .. 4g + 3)
-        const uint32_t* src = p.words + (static_cast<int64_t>(ia) + ipos + 4 * lane);
-        const uint32_t dst = stage + static_cast<uint32_t>(slot * kBatchWords * 4 + lane * 16);
-        if (4 * lane < cnt) cp_async_16(dst, src);
-        if (4 * (lane + 32) < cnt) cp_async_16(dst + 512, src + 128);
-        ipos += kBatchWords;
-        if (ipos >= in) {
-          flags |= kDescLast;
-          ++ij;
-          ipos = 0;
-        }
-        desc = static_cast<uint32_t>(cnt) | ((itile & kDescTileMask) << kDescTileShift) | flags;
-      } else {
-        desc = 0u;
+    auto validate = [&](int32_t& ta, int32_t& tb) {
+      const int32_t n = tb - ta;
+      const bool ok = ta >= 0 && n >= 0 && !(ta & 3) && !(n & 3) && n <= kMaxTileWords && tb <= p.nwords;
+      if (!ok) {
+        record_status(p.status, FLASHSPMM_ERR_CORRUPT_FORMAT);
+        ta = 0;
+        tb = 0;
       }
-      cp_async_commit();  // one group per batch slot, empty ones included, so the counting stays uniform
     };
-
-    // ---- expand side
-    int pj = 0;  // index (among this pair's steps) of the step being expanded
-    auto process = [&](uint32_t desc, int slot) -> bool {
-      if (desc & kDescFirst) {
-        // the buffer is free once the MMAs of its previous step have retired
-        if (!mbar_wait(&empty[pair], static_cast<uint32_t>((pj & 1) ^ 1), abort_flag, budget, p.status)) return false;
-        if (h == 0 && lane == 0) {
-          // the step's B slab: 64 K values x N_MMA rows (rows past N read as zero)
-          mbar_expect_tx(&full[pair], static_cast<uint32_t>(Cf::kBSlabBytes));
-          tma_load_2d(pbuf + kDenseBytes, &tmap_b, static_cast<int32_t>((desc >> kDescTileShift) & kDescTileMask) * kTile,
-                      0, &full[pair]);
-        }
+    int32_t ca, cb, na, nb;
+    int tab_base = 0, ik = 0;  // steps of this warp: at most a piece's steps, far below 2^31
+    uint32_t ipos = 0;
+    const int my_steps32 = static_cast<int>(my_steps);
+    load_tab(0, ca, cb);
+    load_tab(32, na, nb);
+    validate(ca, cb);
+    auto issue = [&](uint32_t (&v)[kRoundRegs], Round& rd) {
+      rd.valid = ik < my_steps32;
+      if (!rd.valid) return;
+      if (ik - tab_base == 32) {
+        tab_base += 32;
+        ca = na;
+        cb = nb;
+        validate(ca, cb);
+        load_tab(tab_base + 32, na, nb);
+      }
+      const int li = ik - tab_base;
+      const uint32_t a0 = static_cast<uint32_t>(__shfl_sync(0xFFFFFFFFu, ca, li));
+      const uint32_t a1 = static_cast<uint32_t>(__shfl_sync(0xFFFFFFFFu, cb, li));
+      const uint32_t base = a0 + ipos;
+      const int rem = min(static_cast<int>(a1 - base), kRoundWords);
+      rd.k = ik;
+      rd.first = ipos == 0;
+      rd.last = base + kRoundWords >= a1;
+      // lane l holds words base + l + 32 i, i < nvalid
+      const int nvalid = rem > lane ? (rem - lane + 31) >> 5 : 0;
+      const uint32_t* src = p.words + base + lane;
 #pragma unroll
-        for (int i = 0; i < kHalfBytes / 16 / 32; ++i) st_shared_zero16(hb + static_cast<uint32_t>((i * 32 + lane) * 16));
+      for (int i = 0; i < kRoundRegs; ++i) v[i] = ldg_word(src + 32 * i, i, nvalid, policy);
+      if (rd.last) {
+        ++ik;
+        ipos = 0;
+      } else {
+        ipos += kRoundWords;
+      }
+    };
+    // Buffer set k & 1 is free once the MMAs of group k - 2 have retired.
+    auto wait_set = [&](int k) -> bool {  // every lane tests the barrier: no broadcast needed
+      return mbar_wait(&a_empty[k & 1], static_cast<uint32_t>(((k >> 1) & 1) ^ 1), abort_flag, budget, p.status);
+    };
+    auto process = [&](const uint32_t (&v)[kRoundRegs], const Round& rd) -> bool {
+      const int set = static_cast<int>(rd.k & 1);
+      uint8_t* half = dense + (pair + kPairs * set) * kDenseBytes + h * kHalfBytes;
+      if (rd.first) {
+        if (!wait_set(rd.k)) return false;
+        uint4* dz = reinterpret_cast<uint4*>(half);
+#pragma unroll
+        for (int i = 0; i < kHalfBytes / 16 / 32; ++i) dz[i * 32 + lane] = make_uint4(0, 0, 0, 0);
         __syncwarp();
       }
-      const int cnt = static_cast<int>(desc & kDescCountMask);
-      const uint32_t* sw = stage_w + slot * kBatchWords + lane;
-      if (cnt == kBatchWords) {
+      const uint32_t hb = smem_u32(half);
 #pragma unroll
-        for (int i = 0; i < kRB; ++i) scatter_word(hb, sw[32 * i]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < kRB; ++i)
-          if (32 * i < cnt) scatter_word(hb, 32 * i + lane < cnt ? sw[32 * i] : kSentinel);
-      }
-      if (desc & kDescLast) {
-        fence_proxy_async_smem();  // generic-proxy stores -> tensor-core (async proxy) reads
+      for (int i = 0; i < kRoundRegs; ++i) scatter_word(hb, v[i]);
+      if (rd.last) {
+        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&full[pair]);
-        ++pj;
+        if (lane == 0) mbar_arrive(&a_full[set]);
       }
       return true;
     };
-
-    uint32_t dsc[kStage];
-#pragma unroll
-    for (int s = 0; s < kStage - 1; ++s) issue(dsc[s], s);
-    bool run = true;
-    while (run) {
-#pragma unroll
-      for (int s = 0; s < kStage; ++s) {
-        if (run) {
-          __syncwarp();  // every lane is done reading the slot about to be refilled
-          issue(dsc[(s + kStage - 1) % kStage], (s + kStage - 1) % kStage);
-          cp_async_wait<kStage - 1>();  // this lane's copies of slot s have landed
-          __syncwarp();                 // ... and every other lane's
-          if (!(dsc[s] & kDescValid) || !process(dsc[s], s)) run = false;
-        }
-      }
+    uint32_t va[kRoundRegs], vb[kRoundRegs];
+    Round ra, rb;
+    bool ok = true;
+    issue(va, ra);
+    while (ra.valid) {
+      issue(vb, rb);
+      if (!(ok = process(va, ra)) || !rb.valid) break;
+      issue(va, ra);
+      if (!(ok = process(vb, rb))) break;
     }
-    cp_async_wait<0>();  // no copy into shared memory outlives the CTA
-    // every B slab this pair requested has landed before shared memory is
-    // released (its last step's full barrier phase completed, or the wait ran
-    // out of budget)
-    if (h == 0 && lane == 0 && pj > 0) mbar_wait_drain(&full[pair], static_cast<uint32_t>((pj - 1) & 1), budget, p.status);
+    // A pair without a step in the piece's last (partial) group still
+    // completes that group's arrival count, once the set is free (so the
+    // arrival cannot count towards the set's previous group).
+    const int64_t ngroups = (piece_steps + kPairs - 1) / kPairs;
+    if (ok && my_steps < ngroups && wait_set(my_steps32)) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[my_steps32 & 1]);
+    }
   }
 
   tc_fence_before_sync();
@@ -622,33 +587,51 @@ EncodeTiledFn get_encode_tiled() {
 template <int N_MMA>
 flashspmm_status launch_bucket(const flashspmm_tcsl* A, const void* B, void* C, int32_t M, int32_t K, int32_t N,
                                const SpmmPlan& plan, void* workspace, cudaStream_t s) {
-  constexpr int ND = Bufs<N_MMA>::value;
-  using Cf = Cfg<N_MMA, ND>;
+  using Cf = Cfg<N_MMA>;
   EncodeTiledFn encode = get_encode_tiled();
   if (!encode) return FLASHSPMM_ERR_CUDA;
-  // B (K x N column-major, i.e. N rows of K) as a 2-D tensor; one request
-  // loads one 64-wide K tile of N_MMA rows, and elements past K or N read as
-  // zero.
+  // B as a 3-D tensor (64 x N x K/64) lets one TMA request load several
+  // consecutive K tiles; a ragged K keeps the 2-D map (one tile per request)
+  // so no box element can fall past the end of B.
+  const int TK = (K + kTile - 1) / kTile;
+  const bool b3d = (K % kTile == 0) && Cf::kSlabsPerReq > 1 && TK >= Cf::kSlabsPerReq;
   CUtensorMap tmap;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTile), static_cast<cuuint32_t>(N_MMA)};
-  const cuuint32_t estride[2] = {1, 1};
-  const CUresult rc = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(B), dims, strides, box,
-                             estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult rc;
+  if (b3d) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kTile), static_cast<cuuint64_t>(N),
+                                static_cast<cuuint64_t>(TK)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2, static_cast<cuuint64_t>(kTile) * 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kTile), static_cast<cuuint32_t>(N_MMA),
+                               static_cast<cuuint32_t>(Cf::kSlabsPerReq)};
+    const cuuint32_t estride[3] = {1, 1, 1};
+    rc = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(B), dims, strides, box, estride,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTile), static_cast<cuuint32_t>(N_MMA)};
+    const cuuint32_t estride[2] = {1, 1};
+    rc = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(B), dims, strides, box, estride,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
   if (rc != CUDA_SUCCESS) return FLASHSPMM_ERR_CUDA;
 
-  auto kernel = spmm_lscd_sm100_kernel<N_MMA, ND>;
   static std::atomic<uint64_t> attr_set_mask{0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FLASHSPMM_ERR_CUDA;
   const uint64_t bit = uint64_t(1) << (dev & 63);
   if (!(attr_set_mask.load() & bit)) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(spmm_lscd_sm100_kernel<N_MMA, kRoundRegsLarge>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(spmm_lscd_sm100_kernel<N_MMA, kRoundRegsSmall>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytes) != cudaSuccess)
       return FLASHSPMM_ERR_CUDA;
     attr_set_mask.fetch_or(bit);
   }
+  const int64_t num_tiles = static_cast<int64_t>(plan.TM) * plan.TK;
+  const bool small_rounds = num_tiles > 0 && A->nwords <= static_cast<int64_t>(kSmallRoundMaxWords) * num_tiles;
 
   SpmmParams p{};
   p.tile_offsets = A->tile_offsets;
@@ -661,6 +644,8 @@ flashspmm_status launch_bucket(const flashspmm_tcsl* A, const void* B, void* C, 
   p.M = M; p.K = K; p.N = N;
   p.TM = plan.TM; p.TK = plan.TK; p.U = plan.U; p.T = plan.T;
   p.mode = plan.mode; p.split = plan.split; p.num_pieces = plan.num_pieces;
+  p.b_kb = b3d ? Cf::kSlabsPerReq : 1;
+  p.b_3d = b3d ? 1 : 0;
   p.timeout_ns = 1000000000ull;  // 1 s: far above any legitimate wait
   p.status = device_status_ptr();
 
@@ -676,7 +661,7 @@ flashspmm_status launch_bucket(const flashspmm_tcsl* A, const void* B, void* C, 
   // the stream; the kernel reads no global memory before griddepcontrol.wait.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(plan.num_pieces));
-  cfg.blockDim = dim3(Cf::kThreads);
+  cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = Cf::kSmemBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -684,7 +669,9 @@ flashspmm_status launch_bucket(const flashspmm_tcsl* A, const void* B, void* C, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, tmap, p);
+  const cudaError_t err =
+      small_rounds ? cudaLaunchKernelEx(&cfg, spmm_lscd_sm100_kernel<N_MMA, kRoundRegsSmall>, tmap, p)
+                   : cudaLaunchKernelEx(&cfg, spmm_lscd_sm100_kernel<N_MMA, kRoundRegsLarge>, tmap, p);
   note_launch();
   return err == cudaSuccess ? FLASHSPMM_OK : FLASHSPMM_ERR_CUDA;
 }
@@ -754,7 +741,6 @@ static bool plan_args_ok(int32_t M, int32_t K, int32_t N, int32_t num_sms) {
 
 flashspmm_status launch_spmm_lscd(const flashspmm_tcsl* A, const void* B, void* C, int32_t M, int32_t K,
                                   int32_t N, const SpmmPlan& plan, void* workspace, cudaStream_t s) {
-  if (static_cast<int64_t>(plan.TK) > kMaxKTiles) return FLASHSPMM_ERR_UNSUPPORTED;
   if (N <= 16) return launch_bucket<16>(A, B, C, M, K, N, plan, workspace, s);
   if (N <= 32) return launch_bucket<32>(A, B, C, M, K, N, plan, workspace, s);
   if (N <= 64) return launch_bucket<64>(A, B, C, M, K, N, plan, workspace, s);
