@@ -53,6 +53,8 @@ def parse_args(argv=None):
     ap.add_argument("--case", default=None,
                     help="single SpMM 'M,K,N,sparsity_pct[,structure]' instead of the layer workload")
     ap.add_argument("--split-k", type=int, default=0)
+    ap.add_argument("--word-order", type=int, default=1, choices=[0, 1],
+                    help="Tiled-CSL word order inside a tile: 0 ascending loc, 1 bank-balanced (v2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0, help="target CPU time of the oracle sample")
@@ -222,6 +224,17 @@ def measured_peaks():
 
 # ---------------------------------------------------------------- oracle (CPU) legs
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def oracle_sample(problems, target_s: float):
     """Time the oracle on the first R rows of every problem (same R for all).
     R starts at 64 and grows (per-call costs make the time far from linear in
@@ -249,9 +262,19 @@ def oracle_sample(problems, target_s: float):
         grow = max(2.0, min(8.0, target_s / max(t, 1e-3)))
         rows = min(max_rows, max(rows + 64, int(rows * grow) // 64 * 64))
         t, nbytes = run(rows)
+    # the same oracle on one thread, on a sample a sixteenth as tall (bounded time)
+    rows1 = max(64, rows // 16 // 64 * 64)
+    nthreads_all = nthreads
+    nthreads = 1
+    t1, nbytes1 = run(min(rows1, max_rows))
+    nthreads = nthreads_all
     return {"value": nbytes / t / 1e9, "unit": "GB/s", "cores": nthreads, "kind": "oracle",
             "sample": f"first {rows} rows of each of the {len(problems)} weight matrices, all N "
-                      f"({nbytes / 1e6:.1f} MB algorithmic, {t:.1f} s)", "rows": rows, "seconds": t}
+                      f"({nbytes / 1e6:.1f} MB algorithmic, {t:.1f} s)", "rows": rows, "seconds": t,
+            "single_thread": {"value": nbytes1 / t1 / 1e9, "unit": "GB/s", "cores": 1,
+                              "sample": f"first {min(rows1, max_rows)} rows of each weight matrix, all N "
+                                        f"({nbytes1 / 1e6:.1f} MB algorithmic, {t1:.1f} s)"},
+            "cpu_model": cpu_model()}
 
 
 def run_reference(args, calls, cfg_name, rank, world):
@@ -312,7 +335,9 @@ def bench_line(*, world, args, cfg_name, work, calls, value, total_ms, tflops, a
                    "sparsity_pct": sorted({c[4] for c in calls}), "split_k": args.split_k,
                    "calls_per_step": len(work),
                    "l2": l2_note(work),
-                   "launch": "one CUDA graph per call, replayed back to back"},
+                   "word_order": "bank-balanced (v2)" if args.word_order else "ascending loc",
+                   "launch": "one CUDA graph per step: the step's SpMM kernels back to back, chained by "
+                             "programmatic dependent launch"},
         "effective_tflops": round(tflops, 3),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": profiled_traffic(cfg_name),
@@ -378,7 +403,7 @@ def main(argv=None):
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        t = fs.tcsl_encode(Wd)
+        t = fs.tcsl_encode(Wd, order=args.word_order)
         e1.record()
         torch.cuda.synchronize()
         fs.check_device_status()
@@ -398,7 +423,10 @@ def main(argv=None):
         ws_need = max(ws_need, fs.spmm_workspace_bytes(M, K, N, args.split_k))
     ws = torch.zeros(max(ws_need, 256), dtype=torch.uint8, device=dev)
 
-    # ---- one CUDA graph per call (memset of arrival counters + the kernel)
+    # ---- one CUDA graph per step: the step's SpMM launches back to back, each
+    # launched with programmatic stream serialisation so its prologue overlaps
+    # the previous kernel's tail.  (One graph per call is also captured, to time
+    # the calls one by one for the per-call detail.)
     stream = torch.cuda.Stream(device=dev)
     for w in work:  # eager warm-up resolves every lazy initialisation outside capture
         with torch.cuda.stream(stream):
@@ -406,23 +434,26 @@ def main(argv=None):
     stream.synchronize()
     fs.check_device_status(stream)
     launches_before = fs.launch_count()
+    step_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(step_graph, stream=stream, capture_error_mode="thread_local"):
+        for w in work:
+            fs.spmm_lscd(w["t"], w["B"], w["C"], split_k=args.split_k, workspace=ws)
+    kernels_per_step = fs.launch_count() - launches_before
     graphs = []
     for w in work:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
             fs.spmm_lscd(w["t"], w["B"], w["C"], split_k=args.split_k, workspace=ws)
         graphs.append(g)
-    kernels_per_step = fs.launch_count() - launches_before
 
     sampler = ClockSampler(dev.index)
     sampler.start()
     time.sleep(0.3)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            for g in graphs:
-                g.replay()
+            step_graph.replay()
     stream.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -430,9 +461,8 @@ def main(argv=None):
     with torch.cuda.stream(stream):
         for k in range(args.steps):
             ev[k][0].record(stream)
-            for i, g in enumerate(graphs):
-                g.replay()
-                ev[k][i + 1].record(stream)
+            step_graph.replay()
+            ev[k][1].record(stream)
     stream.synchronize()
     torch.cuda.synchronize()
     t_wall1 = time.time()
@@ -442,18 +472,29 @@ def main(argv=None):
     sampler.stop()
     clocks = sampler.summary(t_wall0 - 0.05, t_wall1 + 0.05)
     fs.check_device_status(stream)
+    step_ms = np.array([ev[k][0].elapsed_time(ev[k][1]) for k in range(args.steps)])
 
-    per_call_ms = np.array([[ev[k][i].elapsed_time(ev[k][i + 1]) for i in range(len(graphs))]
-                            for k in range(args.steps)])
-    step_ms = np.array([ev[k][0].elapsed_time(ev[k][-1]) for k in range(args.steps)])
+    # per-call detail (outside the timed region): each call's graph, timed one by one
+    reps = max(3, min(args.steps, 10))
+    cev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)] for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        for k in range(reps):
+            cev[k][0].record(stream)
+            for i, g in enumerate(graphs):
+                g.replay()
+                cev[k][i + 1].record(stream)
+    stream.synchronize()
+    fs.check_device_status(stream)
+    per_call_ms = np.array([[cev[k][i].elapsed_time(cev[k][i + 1]) for i in range(len(graphs))]
+                            for k in range(reps)])
     total_ms = max_over_ranks(float(step_ms.sum()), world, dev)
     bytes_step = sum(w["bytes"] for w in work)
     flops_step = sum(w["flops"] for w in work)
     value = job_throughput(bytes_step, args.steps, total_ms, world)
     tflops = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
     peak, peak_src = measured_peaks()
-    kernel_ms = float(per_call_ms.sum())
-    achieved = bytes_step * args.steps / (kernel_ms * 1e-3) / 1e9
+    # the step is the path's kernels back to back: its device time is the kernels' time
+    achieved = bytes_step * args.steps / (float(step_ms.sum()) * 1e-3) / 1e9
 
     detail = []
     for i, w in enumerate(work):

@@ -244,6 +244,24 @@ int flashspmm_plan_query(int32_t M, int32_t K, int32_t N, int32_t split_k, int32
 int64_t flashspmm_plan_owner(int32_t M, int32_t K, int32_t N, int32_t split_k, int32_t num_sms, int64_t q);
 int64_t flashspmm_plan_slot(int32_t M, int32_t K, int32_t N, int32_t split_k, int32_t num_sms, int64_t pc, int64_t u);
 
+/* Dense or sparse, per MatMul [lscd] (the Flash-LLM review, section 5 item 5:
+ * the integration's GEMM wrapper picks dense or sparse per weight; section 6,
+ * "N dimension": the sparse kernel wins only for skinny N).  From time models
+ * fitted to this library's SpMM and to dense fp16 cuBLAS GEMMs of the same
+ * shapes on B200 (inputs resident in HBM, CUDA-graph launches):
+ *   flashspmm_predict_us     predicted microseconds of this library's SpMM
+ *                            (automatic split) and of a dense GEMM for an
+ *                            M x K weight with nnz stored entries and N
+ *                            columns on num_sms SMs; 0, or -1 on bad
+ *                            arguments (M, K, N, num_sms > 0, N <= 256,
+ *                            nnz >= 0).  Either output pointer may be NULL.
+ *   flashspmm_prefer_sparse  1 when the SpMM is predicted faster, 0 when the
+ *                            dense GEMM is, -1 on bad arguments.
+ * Host only, no device needed; running the dense GEMM stays the caller's job. */
+int flashspmm_predict_us(int32_t M, int32_t K, int32_t N, int64_t nnz, int32_t num_sms, double* t_sparse,
+                         double* t_dense);
+int flashspmm_prefer_sparse(int32_t M, int32_t K, int32_t N, int64_t nnz, int32_t num_sms);
+
 /* Synchronises `stream`, then reads and clears the library's device status
  * word for the current device: FLASHSPMM_OK or the first error a kernel
  * recorded since the last read. */

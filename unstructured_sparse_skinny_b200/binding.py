@@ -65,6 +65,8 @@ def load_library():
         "flashspmm_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, P]),
         "flashspmm_launch_count": (ctypes.c_uint64, []),
         "flashspmm_plan_query": (ctypes.c_int, [I32, I32, I32, I32, I32, P, P]),
+        "flashspmm_predict_us": (ctypes.c_int, [I32, I32, I32, I64, I32, P, P]),
+        "flashspmm_prefer_sparse": (ctypes.c_int, [I32, I32, I32, I64, I32]),
         "flashspmm_plan_owner": (ctypes.c_int64, [I32, I32, I32, I32, I32, ctypes.c_int64]),
         "flashspmm_plan_slot": (ctypes.c_int64, [I32, I32, I32, I32, I32, ctypes.c_int64, ctypes.c_int64]),
     }
@@ -190,6 +192,23 @@ def plan_owner(M: int, K: int, N: int, split_k: int, num_sms: int, q: int) -> in
 
 def plan_slot(M: int, K: int, N: int, split_k: int, num_sms: int, pc: int, u: int) -> int:
     return int(load_library().flashspmm_plan_slot(M, K, N, split_k, num_sms, pc, u))
+
+
+def predict_us(M: int, K: int, N: int, nnz: int, num_sms: int = 148) -> tuple:
+    """(sparse, dense) predicted microseconds of one call (host-side model; see
+    flashspmm_predict_us in include/flashspmm.h)."""
+    a, b = ctypes.c_double(), ctypes.c_double()
+    if load_library().flashspmm_predict_us(M, K, N, nnz, num_sms, ctypes.byref(a), ctypes.byref(b)) != 0:
+        raise FlashSpmmError(1, "predict_us")
+    return a.value, b.value
+
+
+def prefer_sparse(M: int, K: int, N: int, nnz: int, num_sms: int = 148) -> bool:
+    """True when this library's SpMM is predicted faster than a dense GEMM."""
+    r = load_library().flashspmm_prefer_sparse(M, K, N, nnz, num_sms)
+    if r < 0:
+        raise FlashSpmmError(1, "prefer_sparse")
+    return r == 1
 
 
 def spmm_workspace_bytes(M: int, K: int, N: int, split_k: int = 0) -> int:
