@@ -195,23 +195,23 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per step measured by ncu for this workload, from the committed
-    summary, or None when it was taken on a different kernel source."""
+def profiled_traffic(workload: str, word_order: int):
+    """DRAM bytes per step measured by ncu for this workload: the one JSON line
+    starting with `roofline_traffic:` in the committed summary, used only while
+    the kernel sources hash to the value recorded there (else None)."""
     f = ROOT / "profiles" / "spmm_lscd_opt66b_layer_dram_traffic.md"
     if workload != "opt66b_layer" or not f.exists():
         return None
-    vals = {}
     for line in f.read_text().splitlines():
-        if line.startswith("- ") and ":" in line:
-            k, v = line[2:].split(":", 1)
-            vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
-        return None
-    try:
-        return int(vals["dram_bytes_per_step"])
-    except (KeyError, ValueError):
-        return None
+        if line.startswith("roofline_traffic:"):
+            try:
+                rec = json.loads(line.split(":", 1)[1])
+            except ValueError:
+                return None
+            if rec.get("kernel_source_sha256_16") != kernel_source_hash() or rec.get("word_order") != word_order:
+                return None
+            return int(rec["dram_bytes_per_step"])
+    return None
 
 
 def measured_peaks():
@@ -340,7 +340,7 @@ def bench_line(*, world, args, cfg_name, work, calls, value, total_ms, tflops, a
                              "programmatic dependent launch"},
         "effective_tflops": round(tflops, 3),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic(cfg_name),
+                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic(cfg_name, args.word_order),
                      "traffic_unit": "DRAM bytes per step (all calls of the step; ncu)",
                      "algorithmic_bytes_per_step": bytes_step,
                      "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)" if peak_src == "measured"
