@@ -29,10 +29,21 @@
  *     the bank-balanced order; the SpMM accepts either), padded to a multiple
  *     of 4 words with the sentinel 0xFFFF0000; tile_m * tile_k <= 65535;
  *   - tile_offsets: int32[num_tiles + 1], in words, tile_offsets[0] = 0.
- *     The SpMM reads them as absolute indices into `words`, so a view whose
- *     tile_offsets point into a larger matrix's offsets (a run of whole
- *     strips, with that matrix's words and nwords) is a valid operand: this
- *     is how a row-split (tensor-parallel) shard is taken without copying.
+ *
+ * Views (tensor-parallel shards without copying; the Flash-LLM review,
+ * section 5 item 5, distributed inference).  The SpMM reads tile offsets as
+ * absolute indices into `words` and addresses tile (i, j) of its operand as
+ * tile_offsets[i * ld + j], so:
+ *   - rows: a run of whole strips of a larger matrix is the view whose
+ *     tile_offsets point at the run's first tile, with that matrix's ld,
+ *     words and nwords;
+ *   - K range: K tiles [j0, j1) of every strip are the view whose
+ *     tile_offsets point at entry j0, with that matrix's ld (its tiles per
+ *     strip), words and nwords, and K = the range's width.  Tile j1 - 1 of a
+ *     strip ends where tile j1 (or the next strip) begins, so no extra entry
+ *     is needed.
+ * flashspmm_tcsl_validate checks whole matrices only (ld equal to the tiles
+ * per strip and offsets starting at 0).
  *
  * Conventions for every call:
  *   - Array arguments are DEVICE pointers owned by the caller (the only host
@@ -55,7 +66,7 @@
 extern "C" {
 #endif
 
-#define FLASHSPMM_ABI_VERSION 1
+#define FLASHSPMM_ABI_VERSION 2
 
 /* Bytes of the fixed device scratch behind flashspmm_spmm_lscd_noalloc. */
 #define FLASHSPMM_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
@@ -75,12 +86,20 @@ typedef enum {
 /* A read-only view of a Tiled-CSL matrix in device memory.  The library owns
  * nothing it points to. */
 typedef struct {
-  int32_t M, K;                 /* dense shape of A */
+  int32_t M, K;                 /* dense shape of A (of the view) */
   int32_t tile_m, tile_k;       /* format tile; the SpMM kernel needs 64 x 64 */
-  int64_t nnz;                  /* stored entries excluding padding (informational) */
-  int64_t nwords;               /* == tile_offsets[num_tiles] */
-  const int32_t* tile_offsets;  /* device, num_tiles + 1 entries (absolute word indices) */
+  int64_t nnz;                  /* stored entries excluding padding (informational; -1 = not counted) */
+  int64_t nwords;               /* words reachable through `words` (a whole matrix: tile_offsets[num_tiles]) */
+  const int32_t* tile_offsets;  /* device; tile (i, j) spans words [tile_offsets[i*ld + j], tile_offsets[i*ld + j + 1]) */
   const uint32_t* words;        /* device, nwords entries, 16-byte aligned */
+  int64_t offsets_ld;           /* ld above: entries from one strip's first tile to the next strip's.
+                                   0 means ceil(K / tile_k), a whole matrix.  A K-range shard of a
+                                   larger matrix keeps that matrix's ld and points tile_offsets at
+                                   its first K tile (see "Views" above). */
+  const int64_t* piece_bounds;  /* optional, device: word-balanced work partition written by
+                                   flashspmm_tcsl_partition for this view; NULL = even pieces */
+  int32_t bounds_pieces;        /* pieces that table describes (it holds bounds_pieces + 1 entries) */
+  int32_t reserved;             /* must be 0 */
 } flashspmm_tcsl;
 
 /* ABI version of the loaded library (FLASHSPMM_ABI_VERSION at build time). */
@@ -141,11 +160,55 @@ flashspmm_status flashspmm_tcsl_reorder_banks(const int32_t* tile_offsets, uint3
  * each tile holds real words with distinct in-range locs and nonzero value
  * bits, in any order (ascending or bank-balanced), then fewer than four exact
  * sentinels).  Any violation records FLASHSPMM_ERR_CORRUPT_FORMAT in the
- * device status word. */
+ * device status word.  A view with offsets_ld other than 0 or ceil(K/tile_k)
+ * returns FLASHSPMM_ERR_UNSUPPORTED (validate the whole matrix instead). */
 flashspmm_status flashspmm_tcsl_validate(const flashspmm_tcsl* A, void* stream);
 
+/* Pieces (CTAs) of the automatic plan (split_k = 0) for an M x K operand on
+ * num_sms SMs: min(num_sms, ceil(T / 4)) with T = ceil(M / 128) * ceil(K / 64)
+ * steps.  flashspmm_tcsl_partition writes that many pieces plus one entry.
+ * -1 on bad arguments (M, K, num_sms > 0).  Host only. */
+int32_t flashspmm_partition_pieces(int32_t M, int32_t K, int32_t num_sms);
+
+/* Word-balanced work partition for the automatic plan [code-layout].  The
+ * plan cuts the step space (step q = u * ceil(K/64) + j: 128-row unit u, K
+ * tile j) into P pieces of consecutive steps, one CTA each.  Without a table
+ * every piece holds the same number of steps, and a piece over denser rows or
+ * columns takes longer.  This call computes pieces of about equal cost
+ * instead, where a step costs 1024 plus its words (both strips' tiles,
+ * padding included): 1024 words is the fixed per-step cost, measured in word
+ * equivalents on B200.  With c(q) the cost of steps [0, q) and c(T) the total,
+ * bounds[pc] is the smallest q with P * c(q) >= pc * c(T).  The entries are
+ * then raised to at least bounds[pc-1] + 1 (from pc = 1 up) and lowered to at
+ * most bounds[pc+1] - 1 (from pc = P - 1 down), so every piece keeps at least
+ * one step.  bounds[0] = 0 and bounds[P] = T.
+ *   A                view with 64 x 64 tiles (any ld); its offsets are read on
+ *                    the device.
+ *   num_sms          SMs of the device that will run the SpMM; 0 = the
+ *                    current device's.
+ *   bounds           device int64[bounds_capacity]; receives P + 1 entries,
+ *                    P = flashspmm_partition_pieces(M, K, num_sms).
+ * To use it, set A->piece_bounds = bounds and A->bounds_pieces = P.  The SpMM
+ * uses a table only when split_k = 0 and P equals its plan's pieces (P <=
+ * 512); otherwise it cuts even pieces.  A table that is not strictly
+ * increasing from 0 to T makes the SpMM record FLASHSPMM_ERR_CORRUPT_FORMAT
+ * and cut even pieces.  More than 16384 units (M > 2,097,152) or P > 512
+ * returns FLASHSPMM_ERR_UNSUPPORTED; bounds_capacity < P + 1 returns
+ * FLASHSPMM_ERR_CAPACITY. */
+flashspmm_status flashspmm_tcsl_partition(const flashspmm_tcsl* A, int32_t num_sms, int64_t* bounds,
+                                          int32_t bounds_capacity, void* stream);
+
+/* Host diagnostic of flashspmm_tcsl_partition: the same rule, run on the host
+ * over a host copy of a view's offsets (tile (i, j) at tile_offsets[i*ld + j];
+ * offsets_ld 0 = ceil(K/64)), for num_pieces pieces.  Writes num_pieces + 1
+ * entries to the host array `bounds`.  0, or -1 on bad arguments. */
+int flashspmm_partition_host(const int32_t* tile_offsets, int64_t offsets_ld, int32_t M, int32_t K,
+                             int32_t num_pieces, int64_t* bounds);
+
 /* Bytes of workspace flashspmm_spmm_lscd needs on the CURRENT device for this
- * problem (0 when no partial sums are needed).  split_k as below. */
+ * problem (0 when no partial sums are needed).  split_k as below.  With
+ * split_k = 0 the size also covers a word-balanced piece table, whose piece
+ * boundaries may fall anywhere (so with more than one piece it is never 0). */
 size_t flashspmm_spmm_workspace_bytes(int32_t M, int32_t K, int32_t N, int32_t split_k);
 
 /* LSCD SpMM [lscd][core-formulas]: C = A x B.
@@ -185,6 +248,22 @@ size_t flashspmm_spmm_workspace_bytes(int32_t M, int32_t K, int32_t N, int32_t s
 flashspmm_status flashspmm_spmm_lscd(const flashspmm_tcsl* A, const void* B, void* C, int32_t M, int32_t K,
                                      int32_t N, int32_t split_k, void* workspace, size_t workspace_bytes,
                                      void* stream);
+
+/* flashspmm_spmm_lscd with fp32 output: C is device fp32, M x N column-major
+ * (a contiguous [N][M] float array), holding the fp32 accumulators without
+ * the fp16 rounding.  This is the partial product of a K-range shard that a
+ * tensor-parallel caller sums across ranks (an all-reduce) before rounding
+ * once.  Other arguments, workspace rules and errors as flashspmm_spmm_lscd;
+ * K == 0 writes zeros. */
+flashspmm_status flashspmm_spmm_lscd_f32(const flashspmm_tcsl* A, const void* B, float* C, int32_t M, int32_t K,
+                                         int32_t N, int32_t split_k, void* workspace, size_t workspace_bytes,
+                                         void* stream);
+
+/* Rounds n fp32 values to fp16 (round to nearest even, overflow to +-Inf):
+ * the last step of a tensor-parallel K split, once the ranks' fp32 partials
+ * (flashspmm_spmm_lscd_f32) have been summed.  x and y are device arrays of n
+ * elements, 16-byte aligned; they may not overlap. */
+flashspmm_status flashspmm_round_f16(const float* x, void* y, int64_t n, void* stream);
 
 /* End-to-end form of flashspmm_spmm_lscd for callers whose activations live
  * in host memory: on `stream` it copies B from B_host (K x N column-major fp16)

@@ -49,7 +49,7 @@ def test_library_is_built_for_sm100a(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.flashspmm_abi_version() == 1
+    assert lib.flashspmm_abi_version() == 2
     for code in range(9):
         assert lib.flashspmm_status_string(code)
     assert lib.flashspmm_status_string(99) == b"unknown status"
@@ -80,6 +80,11 @@ FAKE = 0x7F0000000000  # never dereferenced: every case below fails a host-side 
     (dict(nwords=6), {}, 6),                   # word count not a multiple of 4
     (dict(tile_offsets=None), {}, 1),          # missing offsets
     (dict(tile_m=256, tile_k=256), {}, 2),     # tile area > 65535
+    (dict(offsets_ld=1), {}, 1),               # offsets ld below the tiles per strip (2)
+    (dict(offsets_ld=-2), {}, 1),              # negative ld
+    (dict(reserved=1), {}, 1),                 # reserved field set
+    (dict(piece_bounds=0x30000), {}, 1),       # a piece table without its piece count
+    (dict(bounds_pieces=-1), {}, 1),           # negative piece count
 ])
 def test_spmm_rejects_bad_arguments(lib, kw, args, status):
     v = _view(**kw)
@@ -87,6 +92,18 @@ def test_spmm_rejects_bad_arguments(lib, kw, args, status):
     a.update(args)
     rc = lib.flashspmm_spmm_lscd(ctypes.byref(v), FAKE, FAKE, a["M"], a["K"], a["N"], 0, None, 0, None)
     assert rc == status
+    rc = lib.flashspmm_spmm_lscd_f32(ctypes.byref(v), FAKE, FAKE, a["M"], a["K"], a["N"], 0, None, 0, None)
+    assert rc == status
+
+
+def test_partition_and_validate_reject_bad_arguments(lib):
+    v = _view()
+    assert lib.flashspmm_tcsl_partition(ctypes.byref(v), 148, None, 8, None) == 1       # no table
+    assert lib.flashspmm_tcsl_partition(ctypes.byref(_view(tile_k=32)), 148, FAKE, 8, None) == 2
+    assert lib.flashspmm_tcsl_partition(ctypes.byref(v), -1, FAKE, 8, None) == 1
+    assert lib.flashspmm_tcsl_validate(ctypes.byref(_view(offsets_ld=4)), None) == 2   # views are not validated
+    assert lib.flashspmm_partition_pieces(0, 64, 148) == -1
+    assert lib.flashspmm_partition_pieces(128, 128, 0) == -1
 
 
 

@@ -27,7 +27,7 @@ def test_gpu_line_has_every_contract_key():
         cpu={"value": 0.15, "unit": "GB/s", "cores": 16, "kind": "oracle", "sample": "rows"},
         e2e={"value": 2088.0, "unit": "GB/s", "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 2},
         kernels_per_step=16, dense=None, clocks={"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []},
-        enc_bytes=10, enc_ms=1.0, detail=[])
+        enc_bytes=10, enc_ms=1.0, enc_first_ms=2.0, detail=[])
     json.dumps(line)
     for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
               "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "cpu_baseline", "e2e",

@@ -7,5 +7,5 @@ streams into the C calls.  There is no CPU fallback: if the library or a CUDA
 device is missing, the calls raise.
 """
 from .binding import (TCSL, FlashSpmmError, check_device_status, launch_count, load_library,  # noqa: F401
-                      predict_us, prefer_sparse, spmm_lscd, spmm_lscd_host, spmm_lscd_noalloc,
-                      spmm_workspace_bytes, tcsl_encode, tcsl_validate)
+                      partition_host, partition_pieces, predict_us, prefer_sparse, spmm_lscd, spmm_lscd_host,
+                      spmm_lscd_noalloc, spmm_workspace_bytes, tcsl_encode, tcsl_validate)

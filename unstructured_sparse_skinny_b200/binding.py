@@ -12,7 +12,7 @@ contiguous ``[N, M]`` tensor (M x N column-major).
 from __future__ import annotations
 
 import ctypes
-from dataclasses import dataclass
+from dataclasses import dataclass, replace
 from pathlib import Path
 
 import torch
@@ -35,7 +35,8 @@ class FlashSpmmError(RuntimeError):
 class _TcslView(ctypes.Structure):
     _fields_ = [("M", ctypes.c_int32), ("K", ctypes.c_int32), ("tile_m", ctypes.c_int32),
                 ("tile_k", ctypes.c_int32), ("nnz", ctypes.c_int64), ("nwords", ctypes.c_int64),
-                ("tile_offsets", ctypes.c_void_p), ("words", ctypes.c_void_p)]
+                ("tile_offsets", ctypes.c_void_p), ("words", ctypes.c_void_p), ("offsets_ld", ctypes.c_int64),
+                ("piece_bounds", ctypes.c_void_p), ("bounds_pieces", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 def load_library():
@@ -59,6 +60,11 @@ def load_library():
         "flashspmm_tcsl_reorder_banks": (ctypes.c_int, [P, P, I64, I32, I32, I32, I32, P]),
         "flashspmm_spmm_workspace_bytes": (SZ, [I32, I32, I32, I32]),
         "flashspmm_spmm_lscd": (ctypes.c_int, [VP, P, P, I32, I32, I32, I32, P, SZ, P]),
+        "flashspmm_spmm_lscd_f32": (ctypes.c_int, [VP, P, P, I32, I32, I32, I32, P, SZ, P]),
+        "flashspmm_partition_pieces": (I32, [I32, I32, I32]),
+        "flashspmm_tcsl_partition": (ctypes.c_int, [VP, I32, P, I32, P]),
+        "flashspmm_partition_host": (ctypes.c_int, [P, I64, I32, I32, I32, P]),
+        "flashspmm_round_f16": (ctypes.c_int, [P, P, I64, P]),
         "flashspmm_spmm_lscd_host": (ctypes.c_int, [VP, P, P, P, P, I32, I32, I32, I32, P, SZ, P]),
         "flashspmm_spmm_lscd_noalloc": (ctypes.c_int, [VP, P, P, I32, I32, I32, I32, P]),
         "flashspmm_get_device_status": (ctypes.c_int, [P]),
@@ -90,52 +96,97 @@ def _stream_handle(stream) -> int:
     return int(stream)
 
 
-_SENTINEL_I32 = -65536  # 0xFFFF0000 as int32: the padding word
-
-
 @dataclass
 class TCSL:
-    """A Tiled-CSL matrix resident in device memory."""
-    tile_offsets: torch.Tensor  # int32 [num_tiles + 1]
+    """A Tiled-CSL matrix resident in device memory, or a view of one."""
+    tile_offsets: torch.Tensor  # int32; tile (i, j) starts at tile_offsets[i * ld + j]
     words: torch.Tensor         # int32 storage of the uint32 words [nwords]
-    nnz: int
+    nnz: int                    # stored entries without padding; -1 for a view (not counted)
     M: int
     K: int
     tile_m: int = 64
     tile_k: int = 64
     order: int = 0              # 0: ascending loc in a tile; 1: bank-balanced (word order v2)
+    offsets_ld: int = 0         # ld above; 0 = ceil(K / tile_k), a whole matrix
+    piece_bounds: torch.Tensor | None = None  # int64 word-balanced piece table (flashspmm_tcsl_partition)
 
     @property
     def nwords(self) -> int:
         return int(self.words.numel())
 
+    @property
+    def ld(self) -> int:
+        return self.offsets_ld or -(-self.K // self.tile_k)
+
     def view(self) -> _TcslView:
+        pb = self.piece_bounds
         return _TcslView(self.M, self.K, self.tile_m, self.tile_k, self.nnz, self.nwords,
-                         self.tile_offsets.data_ptr(), self.words.data_ptr() if self.nwords else None)
+                         self.tile_offsets.data_ptr(), self.words.data_ptr() if self.nwords else None,
+                         self.offsets_ld, pb.data_ptr() if pb is not None else None,
+                         pb.numel() - 1 if pb is not None else 0, 0)
 
     def slice_rows(self, row_begin: int, row_end: int) -> "TCSL":
-        """Rows [row_begin, row_end) as a Tiled-CSL view for row-split (tensor-parallel)
+        """Rows [row_begin, row_end) as a view for row-split (tensor-parallel)
         sharding; nothing is copied.  row_begin must start a strip (a multiple of
         tile_m) and row_end must end one or be M.  The view keeps this matrix's
-        word array: tile offsets are absolute word indices, so the shard's offsets
-        are a slice of the full offsets and every tile finds its words unchanged."""
+        words and ld and points its offsets at the first strip of the range."""
         if not (0 <= row_begin < row_end <= self.M) or row_begin % self.tile_m or \
                 (row_end % self.tile_m and row_end != self.M):
             raise ValueError("a row slice must start and end on strip boundaries")
-        TK = -(-self.K // self.tile_k)
-        i0, i1 = row_begin // self.tile_m, -(-row_end // self.tile_m)
-        offs = self.tile_offsets[i0 * TK:i1 * TK + 1]
-        a, b = (int(x) for x in offs[[0, -1]].tolist())
-        nnz = int((self.words[a:b] != _SENTINEL_I32).sum()) if b > a else 0
-        return TCSL(offs, self.words, nnz, row_end - row_begin, self.K, self.tile_m, self.tile_k, self.order)
+        i0 = row_begin // self.tile_m
+        return replace(self, tile_offsets=self.tile_offsets[i0 * self.ld:], nnz=-1, M=row_end - row_begin,
+                       offsets_ld=self.ld, piece_bounds=None)
+
+    def slice_cols(self, k_begin: int, k_end: int) -> "TCSL":
+        """Columns [k_begin, k_end) of A (K tiles of every strip) as a view for
+        K-split (row-parallel) sharding; nothing is copied.  k_begin must start
+        a K tile and k_end must end one or be K.  The view keeps this matrix's
+        words and ld and points its offsets at K tile k_begin / tile_k."""
+        if not (0 <= k_begin < k_end <= self.K) or k_begin % self.tile_k or \
+                (k_end % self.tile_k and k_end != self.K):
+            raise ValueError("a column slice must start and end on K-tile boundaries")
+        return replace(self, tile_offsets=self.tile_offsets[k_begin // self.tile_k:], nnz=-1, K=k_end - k_begin,
+                       offsets_ld=self.ld, piece_bounds=None)
+
+    def partition(self, num_sms: int = 0, stream=None) -> "TCSL":
+        """This matrix with a word-balanced piece table for the automatic SpMM
+        plan on num_sms SMs (0 = the current device's), computed on the device."""
+        lib = load_library()
+        sms = num_sms or torch.cuda.get_device_properties(self.tile_offsets.device).multi_processor_count
+        P = int(lib.flashspmm_partition_pieces(self.M, self.K, sms))
+        if P < 0:
+            raise FlashSpmmError(1, "partition_pieces")
+        bounds = torch.empty(P + 1, dtype=torch.int64, device=self.tile_offsets.device)
+        plain = replace(self, piece_bounds=None)
+        v = plain.view()
+        _check(lib.flashspmm_tcsl_partition(ctypes.byref(v), sms, bounds.data_ptr(), P + 1,
+                                            _stream_handle(stream)), "tcsl_partition")
+        return replace(self, piece_bounds=bounds)
 
 
-def tcsl_encode(A_dense: torch.Tensor, tile_m: int = 64, tile_k: int = 64, stream=None, order: int = 0) -> TCSL:
+def partition_host(tile_offsets, M: int, K: int, num_pieces: int, offsets_ld: int = 0) -> list:
+    """The partition rule run on the host over a host copy of the offsets
+    (diagnostics and tests; the device computes the same table)."""
+    import numpy as np
+    off = np.ascontiguousarray(np.asarray(tile_offsets, dtype=np.int32))
+    out = (ctypes.c_int64 * (num_pieces + 1))()
+    if load_library().flashspmm_partition_host(off.ctypes.data, offsets_ld, M, K, num_pieces, out) != 0:
+        raise FlashSpmmError(1, "partition_host")
+    return [int(x) for x in out]
+
+
+def partition_pieces(M: int, K: int, num_sms: int) -> int:
+    return int(load_library().flashspmm_partition_pieces(M, K, num_sms))
+
+
+def tcsl_encode(A_dense: torch.Tensor, tile_m: int = 64, tile_k: int = 64, stream=None, order: int = 0,
+                partition: bool = False) -> TCSL:
     """Encode a row-major fp16 ``[M, K]`` device tensor into Tiled-CSL on the GPU.
 
     Runs the count pass, reads the word total back (one host sync), allocates
     the words with torch, then runs the fill pass; ``order=1`` adds the
-    in-place bank-balanced reordering (64 x 64 tiles only)."""
+    in-place bank-balanced reordering and ``partition=True`` the word-balanced
+    piece table for the current device (both 64 x 64 tiles only)."""
     if order not in (0, 1):
         raise ValueError("order must be 0 (ascending loc) or 1 (bank-balanced)")
     lib = load_library()
@@ -159,7 +210,8 @@ def tcsl_encode(A_dense: torch.Tensor, tile_m: int = 64, tile_k: int = 64, strea
     if order == 1:
         _check(lib.flashspmm_tcsl_reorder_banks(off.data_ptr(), words.data_ptr() if nwords else None, nwords, M, K,
                                                 tile_m, tile_k, s), "tcsl_reorder_banks")
-    return TCSL(off, words, int(nnz.item()), M, K, tile_m, tile_k, order)
+    t = TCSL(off, words, int(nnz.item()), M, K, tile_m, tile_k, order)
+    return t.partition(stream=stream) if partition and M > 0 and K > 0 else t
 
 
 def tcsl_validate(A: TCSL, stream=None) -> None:
@@ -233,7 +285,8 @@ def _workspace(device: torch.device, nbytes: int) -> torch.Tensor | None:
 def spmm_lscd(tcsl_A: TCSL, B: torch.Tensor, C: torch.Tensor | None = None, M: int | None = None,
               K: int | None = None, N: int | None = None, split_k: int = 0, stream=None,
               workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """C = A x B.  B is the contiguous ``[N, K]`` fp16 tensor; returns C as ``[N, M]`` fp16."""
+    """C = A x B.  B is the contiguous ``[N, K]`` fp16 tensor; returns C as ``[N, M]`` fp16, or
+    writes the given C, which may be fp32 (the unrounded accumulators: a K-split shard's partial)."""
     lib = load_library()
     M = tcsl_A.M if M is None else M
     K = tcsl_A.K if K is None else K
@@ -244,13 +297,14 @@ def spmm_lscd(tcsl_A: TCSL, B: torch.Tensor, C: torch.Tensor | None = None, M: i
         raise ValueError(f"B has shape {tuple(B.shape)}, expected ({N}, {K})")
     if C is None:
         C = torch.empty((N, M), dtype=torch.float16, device=B.device)
-    elif C.shape != (N, M) or C.dtype != torch.float16 or not C.is_contiguous():
-        raise ValueError("C must be a contiguous [N, M] float16 tensor")
+    elif C.shape != (N, M) or C.dtype not in (torch.float16, torch.float32) or not C.is_contiguous():
+        raise ValueError("C must be a contiguous [N, M] float16 or float32 tensor")
     need = int(lib.flashspmm_spmm_workspace_bytes(M, K, N, split_k))
     if workspace is None:
         workspace = _workspace(B.device, need)
     v = tcsl_A.view()
-    _check(lib.flashspmm_spmm_lscd(ctypes.byref(v), B.data_ptr(), C.data_ptr(), M, K, N, split_k,
+    fn = lib.flashspmm_spmm_lscd if C.dtype == torch.float16 else lib.flashspmm_spmm_lscd_f32
+    _check(fn(ctypes.byref(v), B.data_ptr(), C.data_ptr(), M, K, N, split_k,
                                    workspace.data_ptr() if workspace is not None else None,
                                    workspace.numel() if workspace is not None else 0, _stream_handle(stream)),
            "spmm_lscd")

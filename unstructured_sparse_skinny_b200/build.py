@@ -12,7 +12,7 @@ from pathlib import Path
 
 PKG = Path(__file__).resolve().parent
 ROOT = PKG.parent
-SOURCES = [PKG / "csrc" / f for f in ("flashspmm_api.cu", "tcsl_encode.cu", "spmm_lscd.cu", "spmm_noalloc.cu", "selftest.cu")]
+SOURCES = [PKG / "csrc" / f for f in ("flashspmm_api.cu", "tcsl_encode.cu", "spmm_lscd.cu", "spmm_noalloc.cu", "partition.cu", "round_f16.cu", "selftest.cu")]
 DEPS = SOURCES + [PKG / "csrc" / f for f in ("common.cuh", "sm100_primitives.cuh")] + [ROOT / "include" / "flashspmm.h"]
 LIB = PKG / "libflashspmm.so"
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -3,6 +3,7 @@
 // SpMM_API (section 5, "project structure"), reshaped as a plain C ABI that
 // takes device pointers, sizes and a stream and never allocates.
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include <atomic>
 #include <cstdint>
@@ -97,6 +98,10 @@ flashspmm_status check_view(const flashspmm_tcsl* A) {
   if (A->nwords > 0 && !A->words) return FLASHSPMM_ERR_INVALID_ARG;
   if (A->words && !aligned16(A->words)) return FLASHSPMM_ERR_ALIGNMENT;
   if ((A->nwords & 3) != 0) return FLASHSPMM_ERR_CORRUPT_FORMAT;
+  const int64_t tk = A->tile_k > 0 ? (static_cast<int64_t>(A->K) + A->tile_k - 1) / A->tile_k : 0;
+  if (A->offsets_ld < 0 || (A->offsets_ld > 0 && A->offsets_ld < tk)) return FLASHSPMM_ERR_INVALID_ARG;
+  if (A->reserved != 0 || A->bounds_pieces < 0 || (A->piece_bounds && A->bounds_pieces == 0))
+    return FLASHSPMM_ERR_INVALID_ARG;
   return FLASHSPMM_OK;
 }
 
@@ -173,18 +178,56 @@ flashspmm_status flashspmm_tcsl_reorder_banks(const int32_t* tile_offsets, uint3
 flashspmm_status flashspmm_tcsl_validate(const flashspmm_tcsl* A, void* stream) {
   flashspmm_status st = check_view(A);
   if (st != FLASHSPMM_OK) return st;
+  if (A->offsets_ld != 0 && A->offsets_ld != (static_cast<int64_t>(A->K) + A->tile_k - 1) / A->tile_k)
+    return FLASHSPMM_ERR_UNSUPPORTED;
   if (!have_device()) return FLASHSPMM_ERR_NO_DEVICE;
   return launch_tcsl_validate(A, as_stream(stream)) == cudaSuccess ? FLASHSPMM_OK : FLASHSPMM_ERR_CUDA;
 }
 
 size_t flashspmm_spmm_workspace_bytes(int32_t M, int32_t K, int32_t N, int32_t split_k) {
   if (M <= 0 || K <= 0 || N <= 0 || N > 256) return 0;
-  return make_spmm_plan(M, K, N, split_k, device_sm_count()).workspace_bytes;
+  const int sms = device_sm_count();
+  const size_t even = make_spmm_plan(M, K, N, split_k, sms).workspace_bytes;
+  if (split_k > 0) return even;
+  const size_t table = make_spmm_plan(M, K, N, split_k, sms, true).workspace_bytes;
+  return table > even ? table : even;
 }
 
-flashspmm_status flashspmm_spmm_lscd(const flashspmm_tcsl* A, const void* B, void* C, int32_t M, int32_t K,
-                                     int32_t N, int32_t split_k, void* workspace, size_t workspace_bytes,
-                                     void* stream) {
+int32_t flashspmm_partition_pieces(int32_t M, int32_t K, int32_t num_sms) {
+  if (M <= 0 || K <= 0 || num_sms <= 0) return -1;
+  return make_spmm_plan(M, K, 8, 0, num_sms).num_pieces;
+}
+
+flashspmm_status flashspmm_tcsl_partition(const flashspmm_tcsl* A, int32_t num_sms, int64_t* bounds,
+                                          int32_t bounds_capacity, void* stream) {
+  flashspmm_status st = check_view(A);
+  if (st != FLASHSPMM_OK) return st;
+  if (A->tile_m != 64 || A->tile_k != 64) return FLASHSPMM_ERR_UNSUPPORTED;
+  if (A->M <= 0 || A->K <= 0 || num_sms < 0 || !bounds) return FLASHSPMM_ERR_INVALID_ARG;
+  if (!have_device()) return FLASHSPMM_ERR_NO_DEVICE;
+  const int sms = num_sms > 0 ? num_sms : device_sm_count();
+  if (sms <= 0) return FLASHSPMM_ERR_NO_DEVICE;
+  const int32_t pieces = flashspmm_partition_pieces(A->M, A->K, sms);
+  if (pieces > kMaxTablePieces) return FLASHSPMM_ERR_UNSUPPORTED;  // the SpMM would not use the table
+  if (bounds_capacity < pieces + 1) return FLASHSPMM_ERR_CAPACITY;
+  if ((static_cast<int64_t>(A->M) + 127) / 128 > kMaxPartitionUnits) return FLASHSPMM_ERR_UNSUPPORTED;
+  return launch_tcsl_partition(A, pieces, bounds, as_stream(stream)) == cudaSuccess ? FLASHSPMM_OK
+                                                                                      : FLASHSPMM_ERR_CUDA;
+}
+
+int flashspmm_partition_host(const int32_t* tile_offsets, int64_t offsets_ld, int32_t M, int32_t K,
+                             int32_t num_pieces, int64_t* bounds) {
+  if (!tile_offsets || !bounds || M <= 0 || K <= 0 || num_pieces <= 0 || offsets_ld < 0) return -1;
+  return partition_host(tile_offsets, offsets_ld, M, K, num_pieces, bounds) ? 0 : -1;
+}
+
+}  // extern "C"
+
+namespace flashspmm {
+
+flashspmm_status prepare_spmm(const flashspmm_tcsl* A, const void* B, void* C, bool c_f32, int32_t M, int32_t K,
+                              int32_t N, int32_t split_k, cudaStream_t s, SpmmPlan* plan, bool* done) {
+  *done = true;
   flashspmm_status st = check_view(A);
   if (st != FLASHSPMM_OK) return st;
   if (M < 0 || K < 0 || N < 0 || A->M != M || A->K != K) return FLASHSPMM_ERR_INVALID_ARG;
@@ -193,21 +236,60 @@ flashspmm_status flashspmm_spmm_lscd(const flashspmm_tcsl* A, const void* B, voi
   if (M == 0 || N == 0) return FLASHSPMM_OK;
   if (!C) return FLASHSPMM_ERR_INVALID_ARG;
   if (!have_device()) return FLASHSPMM_ERR_NO_DEVICE;
-  cudaStream_t s = as_stream(stream);
   if (K == 0) {
-    return cudaMemsetAsync(C, 0, static_cast<size_t>(M) * N * 2, s) == cudaSuccess ? FLASHSPMM_OK
-                                                                                    : FLASHSPMM_ERR_CUDA;
+    const size_t bytes = static_cast<size_t>(M) * N * (c_f32 ? 4 : 2);
+    return cudaMemsetAsync(C, 0, bytes, s) == cudaSuccess ? FLASHSPMM_OK : FLASHSPMM_ERR_CUDA;
   }
   if (!B) return FLASHSPMM_ERR_INVALID_ARG;
   if (!aligned16(B)) return FLASHSPMM_ERR_ALIGNMENT;
   const int sms = device_sm_count();
   if (sms <= 0) return FLASHSPMM_ERR_NO_DEVICE;
-  const SpmmPlan plan = make_spmm_plan(M, K, N, split_k, sms);
+  *plan = make_spmm_plan(M, K, N, split_k, sms);
+  // a piece table is used when it was made for exactly this plan's pieces
+  if (split_k <= 0 && A->piece_bounds && A->bounds_pieces == plan->num_pieces)
+    *plan = make_spmm_plan(M, K, N, split_k, sms, true);
+  *done = false;
+  return FLASHSPMM_OK;
+}
+
+}  // namespace flashspmm
+
+extern "C" {
+
+static flashspmm_status spmm_with_workspace(const flashspmm_tcsl* A, const void* B, void* C, bool c_f32, int32_t M,
+                                            int32_t K, int32_t N, int32_t split_k, void* workspace,
+                                            size_t workspace_bytes, void* stream) {
+  cudaStream_t s = as_stream(stream);
+  SpmmPlan plan{};
+  bool done = true;
+  const flashspmm_status st = prepare_spmm(A, B, C, c_f32, M, K, N, split_k, s, &plan, &done);
+  if (st != FLASHSPMM_OK || done) return st;
   if (plan.workspace_bytes > 0) {
     if (!workspace || workspace_bytes < plan.workspace_bytes) return FLASHSPMM_ERR_CAPACITY;
     if (!aligned16(workspace)) return FLASHSPMM_ERR_ALIGNMENT;
   }
-  return launch_spmm_lscd(A, B, C, M, K, N, plan, workspace, s);
+  return launch_spmm_lscd(A, B, C, c_f32, M, K, N, plan, workspace, s);
+}
+
+flashspmm_status flashspmm_spmm_lscd(const flashspmm_tcsl* A, const void* B, void* C, int32_t M, int32_t K,
+                                     int32_t N, int32_t split_k, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  return spmm_with_workspace(A, B, C, false, M, K, N, split_k, workspace, workspace_bytes, stream);
+}
+
+flashspmm_status flashspmm_spmm_lscd_f32(const flashspmm_tcsl* A, const void* B, float* C, int32_t M, int32_t K,
+                                         int32_t N, int32_t split_k, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  return spmm_with_workspace(A, B, C, true, M, K, N, split_k, workspace, workspace_bytes, stream);
+}
+
+flashspmm_status flashspmm_round_f16(const float* x, void* y, int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return FLASHSPMM_ERR_INVALID_ARG;
+  if (n == 0) return FLASHSPMM_OK;
+  if (!aligned16(x) || !aligned16(y)) return FLASHSPMM_ERR_ALIGNMENT;
+  if (!have_device()) return FLASHSPMM_ERR_NO_DEVICE;
+  return launch_round_f16(x, static_cast<__half*>(y), n, as_stream(stream)) == cudaSuccess ? FLASHSPMM_OK
+                                                                                          : FLASHSPMM_ERR_CUDA;
 }
 
 flashspmm_status flashspmm_spmm_lscd_host(const flashspmm_tcsl* A, const void* B_host, void* C_host, void* B_dev,

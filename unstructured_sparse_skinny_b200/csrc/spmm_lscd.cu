@@ -71,6 +71,7 @@ constexpr int kBarEpi = 1;                          // named barrier id of the e
 constexpr int kRoundRegsLarge = 32, kRoundRegsSmall = 16;
 constexpr int kSmallRoundMaxWords = 448;
 constexpr int kMinStepsPerPiece = 4;
+constexpr int kTableBytes = (kMaxTablePieces + 1) * 8;  // a CTA's checked copy of the piece table
 
 
 template <int N_MMA>
@@ -88,15 +89,17 @@ struct Cfg {
   static constexpr int kOffBars = kOffB + kNumReq * kReqBytes;
   static constexpr int kNumBars = 2 * 2 + 2 * kNumReq + 4 + 1;
   static constexpr int kOffMisc = kOffBars + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
-  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static constexpr int kOffTable = kOffMisc + 64;  // piece-table copy (table instances only)
+  static constexpr int kSmemBytes = kOffTable + 1024;                 // + alignment slack
+  static constexpr int kSmemBytesTable = kOffTable + kTableBytes + 1024;
+  static_assert(kSmemBytesTable <= 232448, "shared memory budget");
 };
 
 struct SpmmParams {
   const int32_t* tile_offsets;
   const uint32_t* words;
   int64_t nwords;
-  __half* C;
+  void* C;           // fp16, or fp32 when c_f32
   float* partials;    // [slot][N][128]
   int32_t* counters;  // mode 0: one per piece (the first piece of a shared unit); mode 1: one per unit
   int32_t M, K, N;
@@ -107,27 +110,47 @@ struct SpmmParams {
   int32_t b_3d;    // B tensor map is 3-D (64 x N x K/64)
   uint64_t timeout_ns;
   int* status;
+  const int64_t* bounds;  // word-balanced piece table (mode 0), or null for even pieces
+  int64_t ld;             // tile_offsets entries between consecutive strips
+  int32_t c_f32;          // C holds fp32 instead of fp16
 };
 
 struct Range {
   int64_t b, e;
 };
 
-__host__ __device__ __forceinline__ Range piece_range(const SpmmParams& p, int64_t pc) {
-  if (p.mode == 0) return {pc * p.T / p.num_pieces, (pc + 1) * p.T / p.num_pieces};
+// First step of piece pc.  `tab` is the CTA's checked copy of a word-balanced
+// piece table (mode 0 only), or null for the closed forms: even pieces of the
+// whole step space (mode 0) or split equal K-chunks per unit (mode 1).
+__host__ __device__ __forceinline__ int64_t piece_begin(const SpmmParams& p, const int64_t* tab, int64_t pc) {
+  if (p.mode == 0) return tab ? tab[pc] : pc * p.T / p.num_pieces;
   const int64_t u = pc / p.split, c = pc - (pc / p.split) * p.split;
-  return {u * p.TK + c * p.TK / p.split, u * p.TK + (c + 1) * p.TK / p.split};
+  return u * p.TK + c * p.TK / p.split;
 }
 
-// Piece that owns step q in mode 0: the largest pc with floor(pc*T/P) <= q.
-__host__ __device__ __forceinline__ int64_t piece_of_step(const SpmmParams& p, int64_t q) {
-  return ((q + 1) * p.num_pieces + p.T - 1) / p.T - 1;
+__host__ __device__ __forceinline__ Range piece_range(const SpmmParams& p, const int64_t* tab, int64_t pc) {
+  return {piece_begin(p, tab, pc), piece_begin(p, tab, pc + 1)};
 }
 
-// Workspace slot of piece pc's partial sum for unit u.
-__host__ __device__ __forceinline__ int64_t partial_slot(const SpmmParams& p, int64_t pc, int64_t u) {
+// Piece that owns step q in mode 0: the largest pc with piece_begin(pc) <= q.
+__host__ __device__ __forceinline__ int64_t piece_of_step(const SpmmParams& p, const int64_t* tab, int64_t q) {
+  if (!tab) return ((q + 1) * p.num_pieces + p.T - 1) / p.T - 1;
+  int64_t lo = 0, hi = p.num_pieces - 1;  // tab[0] = 0 <= q
+  while (lo < hi) {
+    const int64_t mid = (lo + hi + 1) >> 1;
+    if (tab[mid] <= q) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Workspace slot of piece pc's partial sum for unit u: in mode 0 a piece has
+// two, one for the unit it starts in and one for the unit it ends in (the
+// units in between are whole and never shared).
+__host__ __device__ __forceinline__ int64_t partial_slot(const SpmmParams& p, const int64_t* tab, int64_t pc,
+                                                         int64_t u) {
   if (p.mode == 1) return pc;
-  return 2 * pc + ((piece_range(p, pc).b / p.TK) != u ? 1 : 0);
+  return 2 * pc + ((piece_begin(p, tab, pc) / p.TK) != u ? 1 : 0);
 }
 
 __device__ __forceinline__ bool named_barrier_or(uint32_t id, uint32_t nthreads, bool pred) {
@@ -180,6 +203,12 @@ __device__ __forceinline__ void scatter_word(uint32_t half_u32, uint32_t w) {
       "r"(w));
 }
 
+// One element of C: fp16 (round to nearest even), or the fp32 accumulator.
+__device__ __forceinline__ void store_c(const SpmmParams& p, int64_t idx, float x) {
+  if (p.c_f32) static_cast<float*>(p.C)[idx] = x;
+  else static_cast<__half*>(p.C)[idx] = __float2half_rn(x);
+}
+
 // A load round of a decompress warp: words [base, end) of one strip tile,
 // at most 32 * RR of them.
 struct Round {
@@ -187,7 +216,9 @@ struct Round {
   bool first, last, valid;
 };
 
-template <int N_MMA, int RR>
+// kTable: the instance that takes its pieces from a word-balanced table (the
+// plain instance has none of that code and none of its shared memory).
+template <int N_MMA, int RR, bool kTable>
 __global__ void __launch_bounds__(kThreads, 1)
     spmm_lscd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_b, const SpmmParams p) {
   using Cf = Cfg<N_MMA>;
@@ -210,8 +241,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* epi_last = reinterpret_cast<volatile int*>(smem + Cf::kOffMisc + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const Range rg = piece_range(p, blockIdx.x);
   const uint64_t budget = p.timeout_ns;
+  Range rg = piece_range(p, nullptr, blockIdx.x);  // even pieces (closed form; replaced by a table's below)
 
   griddep_launch_dependents();
   if (warp == kWarpB) {
@@ -246,6 +277,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Everything above touched no global memory; from here on the inputs (which
   // the previous kernel in the stream may have written) are read.
   griddep_wait();
+
+  // A word-balanced piece table is copied whole into every CTA and checked
+  // there (strictly increasing from 0 to T), so all CTAs take the same
+  // decision: the table's pieces, or even pieces when it is malformed.
+  const int64_t* tab = nullptr;
+  if (kTable && p.bounds) {
+    int64_t* st = reinterpret_cast<int64_t*>(smem + Cf::kOffTable);
+    const int np = p.num_pieces;  // <= kMaxTablePieces (checked on the host)
+    for (int i = threadIdx.x; i <= np; i += kThreads) st[i] = __ldg(p.bounds + i);
+    __syncthreads();
+    bool bad = false;
+    for (int i = threadIdx.x; i <= np; i += kThreads) {
+      bad |= i == 0 ? st[0] != 0 : st[i] <= st[i - 1];
+      if (i == np) bad |= st[np] != p.T;
+    }
+    if (__syncthreads_or(bad)) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) record_status(p.status, FLASHSPMM_ERR_CORRUPT_FORMAT);
+    } else {
+      tab = st;
+      rg = piece_range(p, tab, blockIdx.x);
+    }
+  }
 
   if (warp == kWarpB) {
     // ------------------------------------------------ dense B producer (TMA)
@@ -372,22 +425,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(ab * N_MMA);
       float* part = nullptr;
-      if (!complete) part = p.partials + partial_slot(p, blockIdx.x, u) * static_cast<int64_t>(p.N) * kUnitRows;
+      if (!complete) part = p.partials + partial_slot(p, tab, blockIdx.x, u) * static_cast<int64_t>(p.N) * kUnitRows;
 #pragma unroll 1
       for (int c = 0; c < N_MMA && c < p.N; c += 16) {
         uint32_t v[16];
         tmem_load_16(taddr + c, v);
         tmem_load_wait();
+        if (!complete) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int nn = c + i;
-          if (nn < p.N) {
-            const float x = __uint_as_float(v[i]);
-            if (complete) {
-              if (m < p.M) p.C[static_cast<int64_t>(nn) * p.M + m] = __float2half_rn(x);
-            } else {
-              part[static_cast<int64_t>(nn) * kUnitRows + row] = x;
-            }
+          for (int i = 0; i < 16; ++i)
+            if (c + i < p.N) part[static_cast<int64_t>(c + i) * kUnitRows + row] = __uint_as_float(v[i]);
+        } else if (m < p.M) {
+          if (p.c_f32) {
+            float* cc = static_cast<float*>(p.C) + m;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (c + i < p.N) cc[static_cast<int64_t>(c + i) * p.M] = __uint_as_float(v[i]);
+          } else {
+            __half* cc = static_cast<__half*>(p.C) + m;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (c + i < p.N) cc[static_cast<int64_t>(c + i) * p.M] = __float2half_rn(__uint_as_float(v[i]));
           }
         }
       }
@@ -398,8 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // last-arriver reduction of the unit's partial sums, in piece order
         int64_t first_pc, ncontrib;
         if (p.mode == 0) {
-          first_pc = piece_of_step(p, u * p.TK);
-          ncontrib = piece_of_step(p, u * p.TK + p.TK - 1) - first_pc + 1;
+          first_pc = piece_of_step(p, tab, u * p.TK);
+          ncontrib = piece_of_step(p, tab, u * p.TK + p.TK - 1) - first_pc + 1;
         } else {
           first_pc = u * p.split;
           ncontrib = p.split;
@@ -418,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
 #pragma unroll 1
             for (int64_t k = 0; k < ncontrib; ++k) {
-              const float* src = p.partials + (partial_slot(p, first_pc + k, u) * p.N + nc) * kUnitRows + row;
+              const float* src = p.partials + (partial_slot(p, tab, first_pc + k, u) * p.N + nc) * kUnitRows + row;
 #pragma unroll
               for (int i = 0; i < 16; ++i)
                 if (nc + i < p.N) acc[i] += __ldcg(src + i * kUnitRows);
@@ -426,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (m < p.M) {
 #pragma unroll
               for (int i = 0; i < 16; ++i)
-                if (nc + i < p.N) p.C[static_cast<int64_t>(nc + i) * p.M + m] = __float2half_rn(acc[i]);
+                if (nc + i < p.N) store_c(p, static_cast<int64_t>(nc + i) * p.M + m, acc[i]);
             }
           }
           if (etid == 0) *counter = 0;  // zero again for the next call
@@ -460,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t u = q / p.TK, j = q - (q / p.TK) * p.TK;
         const int64_t strip = 2 * u + h;
         if (strip < p.TM) {
-          const int64_t t = strip * p.TK + j;
+          const int64_t t = strip * p.ld + j;
           ta = __ldg(p.tile_offsets + t);
           tb = __ldg(p.tile_offsets + t + 1);
         }
@@ -585,8 +643,8 @@ EncodeTiledFn get_encode_tiled() {
 }
 
 template <int N_MMA>
-flashspmm_status launch_bucket(const flashspmm_tcsl* A, const void* B, void* C, int32_t M, int32_t K, int32_t N,
-                               const SpmmPlan& plan, void* workspace, cudaStream_t s) {
+flashspmm_status launch_bucket(const flashspmm_tcsl* A, const void* B, void* C, bool c_f32, int32_t M, int32_t K,
+                               int32_t N, const SpmmPlan& plan, void* workspace, cudaStream_t s) {
   using Cf = Cfg<N_MMA>;
   EncodeTiledFn encode = get_encode_tiled();
   if (!encode) return FLASHSPMM_ERR_CUDA;
@@ -623,10 +681,14 @@ flashspmm_status launch_bucket(const flashspmm_tcsl* A, const void* B, void* C, 
   if (cudaGetDevice(&dev) != cudaSuccess) return FLASHSPMM_ERR_CUDA;
   const uint64_t bit = uint64_t(1) << (dev & 63);
   if (!(attr_set_mask.load() & bit)) {
-    if (cudaFuncSetAttribute(spmm_lscd_sm100_kernel<N_MMA, kRoundRegsLarge>,
+    if (cudaFuncSetAttribute(spmm_lscd_sm100_kernel<N_MMA, kRoundRegsLarge, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(spmm_lscd_sm100_kernel<N_MMA, kRoundRegsSmall>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytes) != cudaSuccess)
+        cudaFuncSetAttribute(spmm_lscd_sm100_kernel<N_MMA, kRoundRegsSmall, false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(spmm_lscd_sm100_kernel<N_MMA, kRoundRegsLarge, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytesTable) != cudaSuccess ||
+        cudaFuncSetAttribute(spmm_lscd_sm100_kernel<N_MMA, kRoundRegsSmall, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytesTable) != cudaSuccess)
       return FLASHSPMM_ERR_CUDA;
     attr_set_mask.fetch_or(bit);
   }
@@ -637,7 +699,10 @@ flashspmm_status launch_bucket(const flashspmm_tcsl* A, const void* B, void* C, 
   p.tile_offsets = A->tile_offsets;
   p.words = A->words;
   p.nwords = A->nwords;
-  p.C = static_cast<__half*>(C);
+  p.C = C;
+  p.c_f32 = c_f32 ? 1 : 0;
+  p.bounds = plan.table ? A->piece_bounds : nullptr;
+  p.ld = A->offsets_ld > 0 ? A->offsets_ld : plan.TK;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   p.partials = plan.partial_bytes ? reinterpret_cast<float*>(ws + plan.partial_offset) : nullptr;
   p.counters = plan.counter_bytes ? reinterpret_cast<int32_t*>(ws + plan.counter_offset) : nullptr;
@@ -662,16 +727,20 @@ flashspmm_status launch_bucket(const flashspmm_tcsl* A, const void* B, void* C, 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(plan.num_pieces));
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = Cf::kSmemBytes;
+  cfg.dynamicSmemBytes = plan.table ? Cf::kSmemBytesTable : Cf::kSmemBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t err =
-      small_rounds ? cudaLaunchKernelEx(&cfg, spmm_lscd_sm100_kernel<N_MMA, kRoundRegsSmall>, tmap, p)
-                   : cudaLaunchKernelEx(&cfg, spmm_lscd_sm100_kernel<N_MMA, kRoundRegsLarge>, tmap, p);
+  cudaError_t err;
+  if (plan.table)
+    err = small_rounds ? cudaLaunchKernelEx(&cfg, spmm_lscd_sm100_kernel<N_MMA, kRoundRegsSmall, true>, tmap, p)
+                       : cudaLaunchKernelEx(&cfg, spmm_lscd_sm100_kernel<N_MMA, kRoundRegsLarge, true>, tmap, p);
+  else
+    err = small_rounds ? cudaLaunchKernelEx(&cfg, spmm_lscd_sm100_kernel<N_MMA, kRoundRegsSmall, false>, tmap, p)
+                       : cudaLaunchKernelEx(&cfg, spmm_lscd_sm100_kernel<N_MMA, kRoundRegsLarge, false>, tmap, p);
   note_launch();
   return err == cudaSuccess ? FLASHSPMM_OK : FLASHSPMM_ERR_CUDA;
 }
@@ -687,7 +756,7 @@ int device_sm_count() {
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-SpmmPlan make_spmm_plan(int32_t M, int32_t K, int32_t N, int32_t split_k, int num_sms) {
+SpmmPlan make_spmm_plan(int32_t M, int32_t K, int32_t N, int32_t split_k, int num_sms, bool table) {
   SpmmPlan pl{};
   pl.TM = (M + kTile - 1) / kTile;
   pl.TK = (K + kTile - 1) / kTile;
@@ -700,8 +769,10 @@ SpmmPlan make_spmm_plan(int32_t M, int32_t K, int32_t N, int32_t split_k, int nu
     const int64_t want = (pl.T + kMinStepsPerPiece - 1) / kMinStepsPerPiece;
     pl.num_pieces = static_cast<int32_t>(max64(1, min64(want, num_sms > 1 ? num_sms : 1)));
     // Partial sums exist only if some piece boundary cuts a unit; the kernel
-    // touches the workspace only for such shared units.
-    bool shared = false;
+    // touches the workspace only for such shared units.  A piece table's
+    // boundaries are known only on the device, so it may cut any unit.
+    pl.table = table && pl.num_pieces <= kMaxTablePieces;
+    bool shared = pl.table && pl.num_pieces > 1;
     for (int64_t pc = 1; pc < pl.num_pieces && !shared; ++pc) shared = (pc * pl.T / pl.num_pieces) % pl.TK != 0;
     pl.partial_slots = shared ? 2 * static_cast<int64_t>(pl.num_pieces) : 0;
   } else {
@@ -739,13 +810,13 @@ static bool plan_args_ok(int32_t M, int32_t K, int32_t N, int32_t num_sms) {
   return M > 0 && K > 0 && N > 0 && N <= 256 && num_sms > 0;
 }
 
-flashspmm_status launch_spmm_lscd(const flashspmm_tcsl* A, const void* B, void* C, int32_t M, int32_t K,
-                                  int32_t N, const SpmmPlan& plan, void* workspace, cudaStream_t s) {
-  if (N <= 16) return launch_bucket<16>(A, B, C, M, K, N, plan, workspace, s);
-  if (N <= 32) return launch_bucket<32>(A, B, C, M, K, N, plan, workspace, s);
-  if (N <= 64) return launch_bucket<64>(A, B, C, M, K, N, plan, workspace, s);
-  if (N <= 128) return launch_bucket<128>(A, B, C, M, K, N, plan, workspace, s);
-  return launch_bucket<256>(A, B, C, M, K, N, plan, workspace, s);
+flashspmm_status launch_spmm_lscd(const flashspmm_tcsl* A, const void* B, void* C, bool c_f32, int32_t M,
+                                  int32_t K, int32_t N, const SpmmPlan& plan, void* workspace, cudaStream_t s) {
+  if (N <= 16) return launch_bucket<16>(A, B, C, c_f32, M, K, N, plan, workspace, s);
+  if (N <= 32) return launch_bucket<32>(A, B, C, c_f32, M, K, N, plan, workspace, s);
+  if (N <= 64) return launch_bucket<64>(A, B, C, c_f32, M, K, N, plan, workspace, s);
+  if (N <= 128) return launch_bucket<128>(A, B, C, c_f32, M, K, N, plan, workspace, s);
+  return launch_bucket<256>(A, B, C, c_f32, M, K, N, plan, workspace, s);
 }
 
 }  // namespace flashspmm
@@ -799,7 +870,7 @@ extern "C" int flashspmm_plan_query(int32_t M, int32_t K, int32_t N, int32_t spl
   if (ranges) {
     const flashspmm::SpmmParams p = flashspmm::plan_params(pl);
     for (int64_t pc = 0; pc < pl.num_pieces; ++pc) {
-      const flashspmm::Range r = flashspmm::piece_range(p, pc);
+      const flashspmm::Range r = flashspmm::piece_range(p, nullptr, pc);
       ranges[2 * pc] = r.b;
       ranges[2 * pc + 1] = r.e;
     }
@@ -812,7 +883,7 @@ extern "C" int64_t flashspmm_plan_owner(int32_t M, int32_t K, int32_t N, int32_t
   if (!flashspmm::plan_args_ok(M, K, N, num_sms)) return -1;
   const flashspmm::SpmmPlan pl = make_spmm_plan(M, K, N, split_k, num_sms);
   if (pl.mode != 0 || q < 0 || q >= pl.T) return -1;
-  return flashspmm::piece_of_step(flashspmm::plan_params(pl), q);
+  return flashspmm::piece_of_step(flashspmm::plan_params(pl), nullptr, q);
 }
 
 extern "C" int64_t flashspmm_plan_slot(int32_t M, int32_t K, int32_t N, int32_t split_k, int32_t num_sms,
@@ -820,5 +891,5 @@ extern "C" int64_t flashspmm_plan_slot(int32_t M, int32_t K, int32_t N, int32_t 
   if (!flashspmm::plan_args_ok(M, K, N, num_sms)) return -1;
   const flashspmm::SpmmPlan pl = make_spmm_plan(M, K, N, split_k, num_sms);
   if (pc < 0 || pc >= pl.num_pieces || u < 0 || u >= pl.U || pl.partial_slots == 0) return -1;
-  return flashspmm::partial_slot(flashspmm::plan_params(pl), pc, u);
+  return flashspmm::partial_slot(flashspmm::plan_params(pl), nullptr, pc, u);
 }

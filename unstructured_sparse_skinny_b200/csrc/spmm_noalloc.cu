@@ -25,8 +25,6 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[FLASHSPMM_NOALLOC_SCR
 // reset makes a new context and so a new lookup.
 void* noalloc_scratch_ptr() { return symbol_address_cached(1, &g_noalloc_scratch); }
 
-bool aligned16_ptr(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 }  // namespace flashspmm
 
@@ -34,26 +32,11 @@ using namespace flashspmm;
 
 extern "C" flashspmm_status flashspmm_spmm_lscd_noalloc(const flashspmm_tcsl* A, const void* B, void* C, int32_t M,
                                                         int32_t K, int32_t N, int32_t split_k, void* stream) {
-  if (!A || M < 0 || K < 0 || N < 0 || A->M != M || A->K != K || A->nwords < 0 || A->nwords > INT32_MAX ||
-      !A->tile_offsets || (A->nwords > 0 && !A->words))
-    return FLASHSPMM_ERR_INVALID_ARG;
-  if (A->tile_m != 64 || A->tile_k != 64 || N > 256 || K % 8 != 0) return FLASHSPMM_ERR_UNSUPPORTED;
-  if (A->words && !aligned16_ptr(A->words)) return FLASHSPMM_ERR_ALIGNMENT;
-  if ((A->nwords & 3) != 0) return FLASHSPMM_ERR_CORRUPT_FORMAT;
-  if (M == 0 || N == 0) return FLASHSPMM_OK;
-  if (!C) return FLASHSPMM_ERR_INVALID_ARG;
-  int ndev = 0;
-  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev <= 0) return FLASHSPMM_ERR_NO_DEVICE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (K == 0) {
-    return cudaMemsetAsync(C, 0, static_cast<size_t>(M) * N * 2, s) == cudaSuccess ? FLASHSPMM_OK
-                                                                                    : FLASHSPMM_ERR_CUDA;
-  }
-  if (!B) return FLASHSPMM_ERR_INVALID_ARG;
-  if (!aligned16_ptr(B)) return FLASHSPMM_ERR_ALIGNMENT;
-  const int sms = device_sm_count();
-  if (sms <= 0) return FLASHSPMM_ERR_NO_DEVICE;
-  const SpmmPlan plan = make_spmm_plan(M, K, N, split_k, sms);
+  SpmmPlan plan{};
+  bool done = true;
+  const flashspmm_status st = prepare_spmm(A, B, C, false, M, K, N, split_k, s, &plan, &done);
+  if (st != FLASHSPMM_OK || done) return st;
   if (plan.workspace_bytes > static_cast<size_t>(FLASHSPMM_NOALLOC_SCRATCH_BYTES)) return FLASHSPMM_ERR_CAPACITY;
   void* scratch = nullptr;
   if (plan.workspace_bytes > 0) {
@@ -67,5 +50,5 @@ extern "C" flashspmm_status flashspmm_spmm_lscd_noalloc(const flashspmm_tcsl* A,
   if (plan.counter_bytes && !plan.counters_cleared &&
       cudaMemsetAsync(static_cast<uint8_t*>(scratch) + plan.counter_offset, 0, plan.counter_bytes, s) != cudaSuccess)
     return FLASHSPMM_ERR_CUDA;
-  return launch_spmm_lscd(A, B, C, M, K, N, plan, scratch, s);
+  return launch_spmm_lscd(A, B, C, false, M, K, N, plan, scratch, s);
 }

@@ -253,7 +253,9 @@ __global__ void __launch_bounds__(kValWarps * 32) tcsl_validate_kernel(const int
 // still holding more than r words are exactly the first k_r ranks, so bank b
 // of rank q places its r-th word at position k_0 + ... + k_{r-1} + q.
 constexpr int kReorderWarps = 2;
-constexpr int kReorderListWords = 4096;
+constexpr int kReorderListWords = 4096;  // longest tile (64 x 64 words)
+constexpr int kBankCap = 128;            // locations per shared-memory bank in a 64 x 64 fp16 tile
+constexpr int kLoadBatch = 4;            // 32-word loads in flight per lane
 
 __device__ __forceinline__ uint32_t word_bank(uint32_t w) {
   const uint32_t x = (w >> 15) & 0x1FFEu;  // 2 * loc for loc < 4096
@@ -263,13 +265,14 @@ __device__ __forceinline__ uint32_t word_bank(uint32_t w) {
 __global__ void __launch_bounds__(kReorderWarps * 32)
     tcsl_reorder_banks_kernel(const int32_t* __restrict__ off, uint32_t* __restrict__ words, int64_t num_tiles,
                               int64_t nwords, int* status) {
-  __shared__ uint32_t s_list[kReorderWarps][kReorderListWords];  // the tile's words grouped by bank
-  __shared__ int s_count[kReorderWarps][32];
+  // A bank of the dense 64 x 64 fp16 tile holds 128 locations, so the tile's
+  // words fit per-bank lists of kBankCap entries; a tile that overflows one
+  // (duplicate locations) is corrupt.
+  __shared__ uint32_t s_list[kReorderWarps][32 * kBankCap];
   __shared__ int s_fill[kReorderWarps][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t lt_mask = (1u << lane) - 1u;
   uint32_t* list = s_list[warp];
-  int* count = s_count[warp];
   int* fill = s_fill[warp];
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kReorderWarps;
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * kReorderWarps + warp; t < num_tiles; t += nwarps) {
@@ -281,60 +284,58 @@ __global__ void __launch_bounds__(kReorderWarps * 32)
     }
     const int len = static_cast<int>(len64);
     uint32_t* tw = words + b0;
-    count[lane] = 0;
     fill[lane] = 0;
     __syncwarp();
-    // pass 1: the real words are those before the first sentinel; count them per bank
+    // One pass, kLoadBatch x 32 words loaded at a time: the real words are
+    // those before the first sentinel; each goes to the end of its bank's
+    // list, in input (ascending loc) order.
     int n = len;
-    bool corrupt = false;
-    for (int i0 = 0; i0 < len; i0 += 32) {
-      const int i = i0 + lane;
-      const uint32_t w = i < len ? tw[i] : kSentinel;
-      const uint32_t sent = __ballot_sync(0xFFFFFFFFu, i < len && w == kSentinel);
-      const int stop = sent ? i0 + __ffs(sent) - 1 : len;
-      const bool real = i < len && i < stop;
-      if (real) {
-        if ((w >> 16) >= 4096u) corrupt = true;
-        else atomicAdd(&count[word_bank(w)], 1);
+    bool corrupt = false, done = false;
+    for (int i0 = 0; i0 < len && !done; i0 += 32 * kLoadBatch) {
+      uint32_t w[kLoadBatch];
+#pragma unroll
+      for (int b = 0; b < kLoadBatch; ++b) {
+        const int i = i0 + 32 * b + lane;
+        w[b] = i < len ? tw[i] : kSentinel;
       }
-      if (sent) {
-        n = stop;
-        break;
+#pragma unroll
+      for (int b = 0; b < kLoadBatch; ++b) {
+        if (done) break;
+        const int j0 = i0 + 32 * b, i = j0 + lane;
+        const uint32_t sent = __ballot_sync(0xFFFFFFFFu, i < len && w[b] == kSentinel);
+        const int stop = sent ? j0 + __ffs(sent) - 1 : len;
+        const bool real = i < len && i < stop;
+        if (real && (w[b] >> 16) >= 4096u) corrupt = true;
+        const uint32_t bank = real ? word_bank(w[b]) : 32u;
+        const uint32_t same = __match_any_sync(0xFFFFFFFFu, bank);
+        const int pos = (real ? fill[bank] : 0) + __popc(same & lt_mask);
+        if (real) {
+          if (pos < kBankCap) list[bank * kBankCap + pos] = w[b];
+          else corrupt = true;
+        }
+        __syncwarp();
+        // the highest lane of each bank group advances that bank's fill
+        if (real && (same >> lane) == 1u) fill[bank] += __popc(same);
+        __syncwarp();
+        if (sent || j0 + 32 >= len) {
+          n = stop;
+          done = true;
+        }
       }
     }
     if (__any_sync(0xFFFFFFFFu, corrupt)) {
       if (lane == 0) record_status(status, FLASHSPMM_ERR_CORRUPT_FORMAT);
       continue;
     }
-    __syncwarp();
-    const int cnt = count[lane];  // lane b: words of bank b
-    int start = cnt;              // exclusive prefix over banks: where bank b's words begin in the list
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xFFFFFFFFu, start, o);
-      if (lane >= o) start += y;
-    }
-    start -= cnt;
-    // pass 2: stable placement of the words into bank-major lists (ascending loc within a bank)
-    for (int i0 = 0; i0 < n; i0 += 32) {
-      const int i = i0 + lane;
-      const bool real = i < n;
-      const uint32_t w = real ? tw[i] : 0u;
-      const uint32_t bank = real ? word_bank(w) : 32u;
-      const uint32_t same = __match_any_sync(0xFFFFFFFFu, bank);
-      const int base = __shfl_sync(0xFFFFFFFFu, start, static_cast<int>(bank & 31u)) + (real ? fill[bank & 31u] : 0);
-      if (real) list[base + __popc(same & lt_mask)] = w;
-      __syncwarp();
-      // the highest lane of each bank group advances that bank's fill
-      if (real && (same >> lane) == 1u) fill[bank] += __popc(same);
-      __syncwarp();
-    }
+    const int cnt = fill[lane];  // lane b: words of bank b
+    const int start = lane * kBankCap;
     // windows
     int taken = 0;  // lane b: words of bank b placed so far
     for (int placed = 0; placed < n;) {
       const int room = min(32, n - placed);
       const int rem = cnt - taken;
       int rank = 0;  // banks with more unplaced words, or as many and a lower index
+#pragma unroll
       for (int l = 0; l < 32; ++l) {
         const int rl = __shfl_sync(0xFFFFFFFFu, rem, l);
         rank += (rl > rem || (rl == rem && l < lane)) ? 1 : 0;
