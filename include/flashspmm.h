@@ -227,10 +227,12 @@ size_t flashspmm_spmm_workspace_bytes(int32_t M, int32_t K, int32_t N, int32_t s
  *   C          device fp16, M x N column-major (a contiguous [N][M] array).
  *   N          1 <= N <= 256.
  *   split_k    0: automatic, the step space (units of 128 rows x 64-wide K
- *              tiles) is cut into one contiguous piece per SM and units shared
- *              by several pieces are reduced by the last CTA to finish
- *              ([code-layout] Reduction kernel, fused here); >= 1: each
- *              128-row unit is cut into min(split_k, ceil(K/64)) K-chunks.
+ *              tiles) is cut into one contiguous piece per SM (even in steps,
+ *              or from A->piece_bounds when it holds a table for this plan,
+ *              see flashspmm_tcsl_partition) and units shared by several
+ *              pieces are reduced by the last CTA to finish ([code-layout]
+ *              Reduction kernel, fused here); >= 1: each 128-row unit is cut
+ *              into min(split_k, ceil(K/64)) K-chunks.
  *              Results are deterministic for a given (problem, split_k, device).
  *   workspace  device, >= flashspmm_spmm_workspace_bytes(...), 16-byte aligned;
  *              may be NULL when that size is 0.  Holds fp32 partial sums and

@@ -179,10 +179,11 @@ def test_workspace_too_small_is_rejected():
 
 @pytest.mark.parametrize("s_pct", [95, 99])
 def test_many_short_tiles_high_sparsity(s_pct):
-    """Large, very sparse problem: every step is a partial one-batch tile, so the
-    decompress warps cycle through their staging slots and buffers far more
-    often than they expand words, and the MMA warps run many rounds per unit
-    (a liveness case: must finish without a timeout, within the bound)."""
+    """Large, very sparse problem: every strip tile is one short load round
+    (the 16-word-round instance), so the decompress warps turn over their two
+    buffer sets far more often than they expand words and the MMA warp issues
+    many groups per unit (a liveness case: must finish without a timeout,
+    within the bound)."""
     W, B = _case(9216, 9216, 8, s_pct, key=(212, s_pct))
     assert_parity(gpu_spmm(gpu_encode(W), B), *_oracle(W, B), f"9216^2 s={s_pct}")
 
